@@ -1,0 +1,372 @@
+#!/usr/bin/env python
+"""Benchmark of block-causal GQA attention on B200.
+
+One step = one pass of the hot path over one synthetic batch: the forward
+(K-hat prologue + K/V tile images, then the attention kernel with the fused Q
+prologue) on the 720p pipelined-inference workload at 24B shape: 4 concurrently
+denoised chunks of 6x45x80 latent tokens (86,400 queries) attending block-causally
+to themselves and to 8 cached chunks (259,200 keys), 128 query / 8 KV heads,
+head_dim 48.  The mask plan is compiled once (host) and reused by every step, as
+every layer of a denoising step reuses it; its compile time is reported apart.
+
+Metric: mask-aware TFLOP/s (4 * D * Hq * visible pairs per forward), whole job.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+N > 1 is launched by torchrun, one rank per GPU; KV groups are split over ranks
+(no data exchange), so total work is fixed ("strong" scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "block-causal attn mask-aware TFLOPS (fwd, fwd+bwd) & % bf16 peak, 1×B200"
+DEFAULT_WORKLOAD = "p720_pipelined"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=8, help="query rows (all heads) in the oracle sample")
+    return ap.parse_args()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples of one GPU while it runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [s for s, p in zip(sm, power) if p > 0.5 * max(power)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+_CPU_INPUTS = {}
+
+
+def _cpu_inputs(w):
+    from block_causal_attention_b200 import workloads as W
+    if w.name not in _CPU_INPUTS:
+        _CPU_INPUTS[w.name] = (W.make_input(w, W.T_K), W.make_input(w, W.T_V),
+                               W.make_input(w, W.T_KC) if w.num_cache_keys else None,
+                               W.make_input(w, W.T_VC) if w.num_cache_keys else None)
+    return _CPU_INPUTS[w.name]
+
+
+def cpu_oracle_sample(w, nrows: int, seed: int):
+    """Time the fp64 oracle (as it stands) on ``nrows`` seeded query rows, all heads.
+    Returns (seconds, mask-aware flops of the sample, description)."""
+    import oracle
+    from block_causal_attention_b200 import workloads as W
+    rows = np.random.default_rng(seed).choice(w.nq, size=nrows, replace=False)
+    rows.sort()
+    k, v, kc, vc = _cpu_inputs(w)
+    q_rows = W.make_input_rows(w, W.T_Q, rows)
+    pairs = sum(int(oracle.mask_row(w.slices_array(), w.nk, int(r)).sum()) for r in rows)
+    t0 = time.perf_counter()
+    oracle.forward(None, k, v, kc, vc, w.videos_array(), w.slices_array(), w.hq, w.hkv, base=w.rope_base,
+                   eps=w.eps, rows=rows, q_rows=q_rows)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * w.d * w.hq * pairs
+    desc = (f"{nrows} seeded query row(s) x all {w.hq} heads of {w.name} ({pairs} visible pairs/head), "
+            f"forward incl. the K prologue of all {w.nq} new keys, fp64")
+    return dt, flops, desc
+
+
+def _cores() -> int:
+    n = os.environ.get("OMP_NUM_THREADS")
+    if n and n.isdigit():
+        return int(n)
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(a):
+    """The reference arm: the fp64 CPU oracle, timed on this host's cores, one
+    bounded row sample of the workload per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from block_causal_attention_b200 import workloads as W
+    w = W.WORKLOADS[a.workload]
+    for s in range(a.warmup):
+        cpu_oracle_sample(w, 1, 100 + s)
+    times, flops = [], []
+    desc = ""
+    for s in range(a.steps):
+        dt, fl, desc = cpu_oracle_sample(w, 1, 200 + s)
+        times.append(dt)
+        flops.append(fl)
+    total_t = sum(times)
+    value = sum(flops) / total_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": a.gpus,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * total_t / a.steps, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "pass": "fwd", "sample_per_step": "1 query row x all heads"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- ours
+
+def run_ours(a):
+    import torch
+    import torch.distributed as dist
+    from block_causal_attention_b200 import Plan, workloads as W
+    from block_causal_attention_b200.sharding import shard_heads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    w = W.WORKLOADS[a.workload]
+    h0, h1, g0, g1 = shard_heads(w.hq, w.hkv, rank, world)
+    hq, hkv = h1 - h0, g1 - g0
+
+    t0 = time.perf_counter()
+    plan = Plan(hq, hkv, w.d, w.videos_array(), w.num_cache_keys, w.slices_array(), w.rope_base, w.eps,
+                w.o_fp32)
+    plan_ms = 1e3 * (time.perf_counter() - t0)
+    info = plan.info()
+
+    def shard(t, a0, a1):
+        return t[:, a0:a1].contiguous() if world > 1 else t
+
+    q = shard(W.make_input(w, W.T_Q, "cuda"), h0, h1)
+    k = shard(W.make_input(w, W.T_K, "cuda"), g0, g1)
+    v = shard(W.make_input(w, W.T_V, "cuda"), g0, g1)
+    kc = shard(W.make_input(w, W.T_KC, "cuda"), g0, g1) if w.num_cache_keys else None
+    vc = shard(W.make_input(w, W.T_VC, "cuda"), g0, g1) if w.num_cache_keys else None
+    o = torch.empty((w.nq, hq, w.d), device="cuda", dtype=torch.float32 if w.o_fp32 else torch.bfloat16)
+    lse = torch.empty((hq, w.nq), device="cuda", dtype=torch.float32)
+    ws = plan.alloc_workspace()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        plan.fwd(q, k, v, kc, vc, o=o, lse=lse, workspace=ws, stream=stream)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(a.warmup):
+        step()
+    barrier()
+    if plan.status() != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    clocks = ClockSampler(gpu_uuid)
+    clocks.start()
+    time.sleep(0.3)
+    plan.profile(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    ev0.record(stream)
+    for _ in range(a.steps):
+        step()
+    ev1.record(stream)
+    barrier()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    prof = plan.profile_read()
+    plan.profile(False)
+    clk = clocks.stop()
+    if plan.status() != 0:
+        raise RuntimeError("device status error in the timed region")
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    pairs = info["visible_pairs"]
+    flops_step_total = 4.0 * w.d * w.hq * pairs           # all ranks together
+    flops_fwd_launch = 4.0 * w.d * hq * pairs            # this rank's launch
+    value = flops_step_total * a.steps / (elapsed_ms * 1e-3) / 1e12
+    tokens_per_s = w.nq * a.steps / (elapsed_ms * 1e-3)
+
+    # ---- end to end through the public API: pinned host inputs -> device -> fwd -> host
+    e2e = None
+    if a.e2e_steps > 0:
+        hq_, hk_, hv_ = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
+        hkc = kc.cpu().pin_memory() if kc is not None else None
+        hvc = vc.cpu().pin_memory() if vc is not None else None
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dkc = torch.empty_like(kc) if kc is not None else None
+        dvc = torch.empty_like(vc) if vc is not None else None
+        h2d = sum(t.numel() * t.element_size() for t in (hq_, hk_, hv_, hkc, hvc) if t is not None)
+        d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+        def e2e_step():
+            dq.copy_(hq_, non_blocking=True)
+            dk.copy_(hk_, non_blocking=True)
+            dv.copy_(hv_, non_blocking=True)
+            if dkc is not None:
+                dkc.copy_(hkc, non_blocking=True)
+                dvc.copy_(hvc, non_blocking=True)
+            plan.fwd(dq, dk, dv, dkc, dvc, o=o, lse=lse, workspace=ws, stream=stream)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(a.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], device="cuda", dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": flops_step_total * a.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e_ms / a.e2e_steps}
+
+    # ---- roofline of the dominant kernel (the attention forward)
+    peaks, peak_src = _peaks()
+    n_fwd, ms_fwd = prof["fwd_kernel"]
+    n_img, ms_img = prof["kv_image_kernel"]
+    avg_fwd_ms = ms_fwd / max(1, n_fwd)
+    achieved = flops_fwd_launch / (avg_fwd_ms * 1e-3) / 1e12
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            traffic = json.load(f).get(f"fwd_kernel:{w.name}")
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
+                "frac": achieved / peak_sus, "traffic": traffic,
+                "kernel": "fwd_kernel", "peak_kind": f"bf16 dense, sustained, {peak_src}",
+                "frac_of_burst_peak": achieved / peak_burst,
+                "kernel_share_of_step": ms_fwd / max(1e-9, ms_fwd + ms_img)}
+
+    # ---- CPU oracle baseline (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        dt, fl, desc = cpu_oracle_sample(w, a.cpu_rows, 1)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle", "sample": desc,
+               "seconds": dt}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": elapsed_ms / a.steps, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "pass": "fwd", "nq": w.nq, "nk": w.nk, "hq": w.hq, "hkv": w.hkv,
+                       "d": w.d, "visible_pairs_per_head": pairs,
+                       "parallelism": f"head-parallel x{world}" if world > 1 else "1 GPU",
+                       "l2": "inputs larger than L2 (Q 1.06 GB, K/V images 0.4 GB, O 1.06 GB)",
+                       "plan_compile_ms": plan_ms, "tokens_per_s": tokens_per_s,
+                       "pct_peak_sustained": 100 * value / peak_sus / world,
+                       "pct_peak_burst": 100 * value / peak_burst / world},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+            "gpu_launches": int(n_fwd + n_img),
+            "kernel_ms": {"fwd_kernel": avg_fwd_ms, "kv_image_kernel": ms_img / max(1, n_img)},
+        }
+        print(json.dumps(line), flush=True)
+    plan.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    a = _args()
+    if a.impl == "reference":
+        return run_reference(a)
+    return run_ours(a)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,1 +1,138 @@
-"""block_causal_attention_b200: block-causal GQA attention for B200 (sm_100a)."""
+"""block_causal_attention_b200: block-causal GQA attention (QK-Norm + 3D RoPE, mask
+given as AttnSlices) for NVIDIA B200 (sm_100a).
+
+The computation lives in libbca.so (C ABI, include/bca.h).  This module only
+marshals arguments: PyTorch provides device memory and streams.  There is no CPU
+or PyTorch fallback: calls fail loudly when the library or a GPU is missing.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import numpy as np
+
+from . import _abi
+from ._abi import BcaError  # noqa: F401
+
+__all__ = ["Plan", "BcaError"]
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else int(t.data_ptr())
+
+
+class Plan:
+    """A compiled block-causal attention problem (mask, schedule, RoPE tables)."""
+
+    def __init__(self, hq: int, hkv: int, d: int, videos, num_cache_keys: int = 0, slices=None,
+                 rope_base=(1e4, 1e4, 1e4), eps: float = 1e-6, o_fp32: bool = False,
+                 host_only: bool = False):
+        flags = (_abi.BCA_O_FP32 if o_fp32 else 0) | (_abi.BCA_PLAN_HOST_ONLY if host_only else 0)
+        prob, keep = _abi.make_problem(hq, hkv, d, videos, num_cache_keys, slices, rope_base, eps, flags)
+        self._lib = _abi.lib()
+        self._h = _abi.ctypes.c_void_p()
+        rc = self._lib.bca_plan_create(_abi.ctypes.byref(prob), _abi.ctypes.byref(self._h))
+        del keep
+        _abi.check(rc, "bca_plan_create")
+        self.hq, self.hkv, self.d = int(hq), int(hkv), int(d)
+        self.o_fp32 = bool(o_fp32)
+        self.host_only = bool(host_only)
+        self.num_cache_keys = int(num_cache_keys)
+        inf = self.info()
+        self.nq, self.nk = inf["num_q"], inf["num_k"]
+        self.device_index = None
+        if not host_only:
+            import torch
+            self.device_index = torch.cuda.current_device()
+
+    @classmethod
+    def from_workload(cls, w, host_only: bool = False, o_fp32: Optional[bool] = None) -> "Plan":
+        return cls(w.hq, w.hkv, w.d, w.videos_array(), w.num_cache_keys, w.slices_array(),
+                   w.rope_base, w.eps, w.o_fp32 if o_fp32 is None else o_fp32, host_only)
+
+    # ------------------------------------------------------------------ host
+    def info(self) -> dict:
+        inf = _abi.bca_plan_info()
+        _abi.check(self._lib.bca_plan_get_info(self._h, _abi.ctypes.byref(inf)), "bca_plan_get_info")
+        return {f: getattr(inf, f) for f, _ in inf._fields_}
+
+    def expand_rows(self, r0: int, r1: int) -> np.ndarray:
+        out = np.zeros((r1 - r0, self.nk), dtype=np.uint8)
+        _abi.check(self._lib.bca_plan_expand_rows(self._h, r0, r1, out.ctypes.data if out.size else None),
+                   "bca_plan_expand_rows")
+        return out
+
+    def workspace_bytes(self, pass_: int = _abi.BCA_PASS_FWD) -> int:
+        return int(self._lib.bca_workspace_bytes(self._h, pass_))
+
+    # ------------------------------------------------------------------ device
+    def _stream(self, stream):
+        import torch
+        if stream is None:
+            stream = torch.cuda.current_stream()
+        return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else stream
+
+    def alloc_workspace(self, pass_: int = _abi.BCA_PASS_FWD):
+        import torch
+        return torch.empty(max(16, self.workspace_bytes(pass_)), dtype=torch.uint8, device="cuda")
+
+    def fwd(self, q, k, v, k_cache=None, v_cache=None, *, o=None, lse=None, workspace=None,
+            q_gain=None, k_gain=None, stream=None):
+        """O [Nq, Hq, D] and LSE [Hq, Nq] for bf16 CUDA tensors q [Nq,Hq,D],
+        k/v [Nq,Hkv,D] and (if the plan has a cache) k_cache/v_cache [Nc,Hkv,D]."""
+        import torch
+        if self.host_only:
+            raise BcaError(_abi.BCA_ERR_HOST_ONLY_PLAN, "fwd")
+        for name, t, rows, heads in (("q", q, self.nq, self.hq), ("k", k, self.nq, self.hkv),
+                                     ("v", v, self.nq, self.hkv)):
+            if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or \
+                    tuple(t.shape) != (rows, heads, self.d):
+                raise ValueError(f"{name}: expected contiguous bf16 CUDA tensor of shape "
+                                 f"{(rows, heads, self.d)}, got {t.dtype} {tuple(t.shape)}")
+        if self.num_cache_keys:
+            for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+                if t is None or t.dtype != torch.bfloat16 or not t.is_contiguous() or \
+                        tuple(t.shape) != (self.num_cache_keys, self.hkv, self.d):
+                    raise ValueError(f"{name}: expected bf16 [{self.num_cache_keys}, {self.hkv}, {self.d}]")
+        dev = q.device
+        if o is None:
+            o = torch.empty((self.nq, self.hq, self.d), device=dev,
+                            dtype=torch.float32 if self.o_fp32 else torch.bfloat16)
+        if lse is None:
+            lse = torch.empty((self.hq, self.nq), device=dev, dtype=torch.float32)
+        if workspace is None:
+            workspace = self.alloc_workspace()
+        rc = self._lib.bca_fwd(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache),
+                               _ptr(q_gain), _ptr(k_gain), _ptr(o), _ptr(lse), _ptr(workspace),
+                               self._stream(stream))
+        _abi.check(rc, "bca_fwd")
+        return o, lse
+
+    def profile(self, enable: bool = True) -> None:
+        """Bracket every kernel launched for this plan with CUDA events."""
+        _abi.check(self._lib.bca_profile_enable(self._h, 1 if enable else 0), "bca_profile_enable")
+
+    def profile_read(self) -> dict:
+        """{kernel name: (launches, total device ms)} since the last read."""
+        out = {}
+        for k, name in _abi.KERNEL_NAMES.items():
+            n = _abi.ctypes.c_int64()
+            ms = _abi.ctypes.c_double()
+            _abi.check(self._lib.bca_profile_read(self._h, k, _abi.ctypes.byref(n), _abi.ctypes.byref(ms)),
+                       "bca_profile_read")
+            out[name] = (int(n.value), float(ms.value))
+        return out
+
+    def status(self, stream=None) -> int:
+        return int(self._lib.bca_status(self._h, self._stream(stream)))
+
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None and self._h.value:
+            self._lib.bca_plan_destroy(self._h)
+            self._h = _abi.ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,247 @@
+// C ABI of libbca.so: argument checks, plan lifetime, launches.  See include/bca.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "kernels.hpp"
+#include "plan.hpp"
+
+struct bca_plan_s {
+    bca::Plan plan;
+};
+
+namespace bca {
+
+ProfScope::ProfScope(Plan &p, int k, cudaStream_t s) : plan(p), kernel(k), stream(s) {
+    if (!plan.profiling) return;
+    if (cudaEventCreate(&start) != cudaSuccess) {
+        start = nullptr;
+        return;
+    }
+    cudaEventRecord(start, stream);
+}
+
+ProfScope::~ProfScope() {
+    if (!start) return;
+    cudaEvent_t stop = nullptr;
+    if (cudaEventCreate(&stop) != cudaSuccess) {
+        cudaEventDestroy(start);
+        return;
+    }
+    cudaEventRecord(stop, stream);
+    plan.prof.push_back({kernel, start, stop});
+}
+
+}  // namespace bca
+
+namespace {
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Upload the plan's tables into one device allocation owned by the plan.
+int upload(bca::Plan &P) {
+    using namespace bca;
+    const size_t s_runoff = round256(P.run_off.size() * sizeof(int32_t));
+    const size_t s_runs = round256(std::max<size_t>(1, P.runs.size()) * sizeof(Run));
+    const size_t s_masks = round256(std::max<size_t>(1, P.masks.size()) * sizeof(uint32_t));
+    const size_t s_items = round256(std::max<size_t>(1, P.items.size()) * sizeof(Item));
+    const size_t s_pos = round256(std::max<size_t>(1, P.pos.size()) * sizeof(uint32_t));
+    const size_t s_rope = round256(std::max<size_t>(1, P.rope.size()) * sizeof(float));
+    const size_t s_status = 256;
+    const size_t total = s_runoff + s_runs + s_masks + s_items + s_pos + s_rope + s_status;
+    if (cudaGetDevice(&P.device) != cudaSuccess) return BCA_ERR_CUDA;
+    void *blob = nullptr;
+    if (cudaMalloc(&blob, total) != cudaSuccess) return BCA_ERR_NO_MEMORY;
+    P.d_blob = blob;
+    uint8_t *b = static_cast<uint8_t *>(blob);
+    size_t off = 0;
+    auto put = [&](const void *src, size_t bytes, size_t slot) -> void * {
+        void *dst = b + off;
+        off += slot;
+        if (bytes && cudaMemcpy(dst, src, bytes, cudaMemcpyHostToDevice) != cudaSuccess) return nullptr;
+        return dst;
+    };
+    P.d_run_off = static_cast<const int32_t *>(put(P.run_off.data(), P.run_off.size() * sizeof(int32_t), s_runoff));
+    P.d_runs = static_cast<const Run *>(put(P.runs.data(), P.runs.size() * sizeof(Run), s_runs));
+    P.d_masks = static_cast<const uint32_t *>(put(P.masks.data(), P.masks.size() * sizeof(uint32_t), s_masks));
+    P.d_items = static_cast<const Item *>(put(P.items.data(), P.items.size() * sizeof(Item), s_items));
+    P.d_pos = static_cast<const uint32_t *>(put(P.pos.data(), P.pos.size() * sizeof(uint32_t), s_pos));
+    P.d_rope = static_cast<const float *>(put(P.rope.data(), P.rope.size() * sizeof(float), s_rope));
+    P.d_status = static_cast<int *>(static_cast<void *>(b + off));
+    if (!P.d_run_off || !P.d_runs || !P.d_masks || !P.d_items || !P.d_pos || !P.d_rope) return BCA_ERR_CUDA;
+    if (cudaMemset(P.d_status, 0, sizeof(int)) != cudaSuccess) return BCA_ERR_CUDA;
+    return BCA_OK;
+}
+
+int check_device(const bca::Plan &P) {
+    if (P.flags & BCA_PLAN_HOST_ONLY) return BCA_ERR_HOST_ONLY_PLAN;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BCA_ERR_CUDA;
+    if (dev != P.device) return BCA_ERR_INVALID_ARGUMENT;
+    return BCA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int bca_plan_create(const bca_problem *problem, bca_plan_t *out) {
+    if (!out) return BCA_ERR_INVALID_ARGUMENT;
+    *out = nullptr;
+    bca_plan_s *h = new (std::nothrow) bca_plan_s();
+    if (!h) return BCA_ERR_NO_MEMORY;
+    int rc = bca::validate_problem(problem, h->plan);
+    if (rc == BCA_OK) {
+        try {
+            rc = bca::compile_plan(h->plan);
+        } catch (const std::bad_alloc &) {
+            rc = BCA_ERR_NO_MEMORY;
+        }
+    }
+    if (rc == BCA_OK && !(h->plan.flags & BCA_PLAN_HOST_ONLY)) rc = upload(h->plan);
+    if (rc != BCA_OK) {
+        bca_plan_destroy(h);
+        return rc;
+    }
+    *out = h;
+    return BCA_OK;
+}
+
+static void drop_profile(bca::Plan &P) {
+    for (auto &r : P.prof) {
+        cudaEventDestroy(static_cast<cudaEvent_t>(r.start));
+        cudaEventDestroy(static_cast<cudaEvent_t>(r.stop));
+    }
+    P.prof.clear();
+}
+
+void bca_plan_destroy(bca_plan_t plan) {
+    if (!plan) return;
+    drop_profile(plan->plan);
+    if (plan->plan.d_blob) {
+        int cur = -1;
+        cudaGetDevice(&cur);
+        if (cur != plan->plan.device) cudaSetDevice(plan->plan.device);
+        cudaFree(plan->plan.d_blob);
+        if (cur >= 0 && cur != plan->plan.device) cudaSetDevice(cur);
+    }
+    delete plan;
+}
+
+int bca_plan_get_info(bca_plan_t plan, bca_plan_info *info) {
+    if (!plan || !info) return BCA_ERR_INVALID_ARGUMENT;
+    const bca::Plan &P = plan->plan;
+    std::memset(info, 0, sizeof(*info));
+    info->num_q = P.nq;
+    info->num_k = P.nk;
+    info->num_cache = P.nc;
+    info->num_q_tiles = P.nqt;
+    info->num_k_tiles = P.nkt;
+    info->num_runs = (int64_t)P.runs.size();
+    info->num_full_tiles = P.nfull;
+    info->num_partial_tiles = P.npartial;
+    info->num_items = (int64_t)P.items.size();
+    info->visible_pairs = P.visible_pairs;
+    info->head_dim_padded = P.dpad;
+    info->tile_q = bca::kTileQ;
+    info->tile_k = bca::kTileK;
+    return BCA_OK;
+}
+
+int bca_plan_expand_rows(bca_plan_t plan, int64_t row_begin, int64_t row_end, uint8_t *out) {
+    if (!plan) return BCA_ERR_INVALID_ARGUMENT;
+    return bca::expand_rows(plan->plan, row_begin, row_end, out);
+}
+
+size_t bca_workspace_bytes(bca_plan_t plan, int pass) {
+    if (!plan) return 0;
+    if (pass == BCA_PASS_FWD) return bca::fwd_workspace_bytes(plan->plan);
+    return 0;
+}
+
+int bca_fwd(bca_plan_t plan, const void *q, const void *k, const void *v, const void *k_cache,
+            const void *v_cache, const float *q_gain, const float *k_gain, void *o, float *lse,
+            void *workspace, void *stream) {
+    if (!plan) return BCA_ERR_INVALID_ARGUMENT;
+    bca::Plan &P = plan->plan;
+    int rc = check_device(P);
+    if (rc != BCA_OK) return rc;
+    if (P.nq == 0) return BCA_OK;
+    if (!q || !k || !v || !o || !lse || !workspace) return BCA_ERR_INVALID_ARGUMENT;
+    if (P.nc > 0 && (!k_cache || !v_cache)) return BCA_ERR_INVALID_ARGUMENT;
+    const void *ptrs[] = {q, k, v, k_cache, v_cache, q_gain, k_gain, o, lse, workspace};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return BCA_ERR_MISALIGNED;
+    bca::FwdIO io{q, k, v, k_cache, v_cache, q_gain, k_gain, o, lse, workspace};
+    return bca::launch_fwd(P, io, static_cast<cudaStream_t>(stream));
+}
+
+int bca_profile_enable(bca_plan_t plan, int enable) {
+    if (!plan) return BCA_ERR_INVALID_ARGUMENT;
+    drop_profile(plan->plan);
+    plan->plan.profiling = enable != 0;
+    return BCA_OK;
+}
+
+int bca_profile_read(bca_plan_t plan, int kernel, int64_t *launches, double *total_ms) {
+    if (!plan || !launches || !total_ms || kernel < 0 || kernel >= BCA_KERNEL_COUNT)
+        return BCA_ERR_INVALID_ARGUMENT;
+    bca::Plan &P = plan->plan;
+    *launches = 0;
+    *total_ms = 0.0;
+    std::vector<bca::Plan::ProfRecord> keep;
+    int rc = BCA_OK;
+    for (auto &r : P.prof) {
+        if (r.kernel != kernel) {
+            keep.push_back(r);
+            continue;
+        }
+        float ms = 0.f;
+        cudaEvent_t a = static_cast<cudaEvent_t>(r.start), b = static_cast<cudaEvent_t>(r.stop);
+        if (cudaEventSynchronize(b) != cudaSuccess || cudaEventElapsedTime(&ms, a, b) != cudaSuccess)
+            rc = BCA_ERR_CUDA;
+        *launches += 1;
+        *total_ms += ms;
+        cudaEventDestroy(a);
+        cudaEventDestroy(b);
+    }
+    P.prof.swap(keep);
+    return rc;
+}
+
+int bca_status(bca_plan_t plan, void *stream) {
+    if (!plan) return BCA_ERR_INVALID_ARGUMENT;
+    const bca::Plan &P = plan->plan;
+    int rc = check_device(P);
+    if (rc != BCA_OK) return rc;
+    int h = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&h, P.d_status, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return BCA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return BCA_ERR_CUDA;
+    if (h == 0) return BCA_OK;
+    if (cudaMemsetAsync(P.d_status, 0, sizeof(int), s) != cudaSuccess) return BCA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return BCA_ERR_CUDA;
+    return (h & bca::kStatusTimeout) ? BCA_ERR_DEVICE_TIMEOUT : BCA_ERR_CUDA;
+}
+
+const char *bca_error_string(int code) {
+    switch (code) {
+        case BCA_OK: return "ok";
+        case BCA_ERR_INVALID_ARGUMENT: return "invalid argument";
+        case BCA_ERR_BAD_SLICE: return "bad AttnSlice (out of range, begin > end, or unknown type)";
+        case BCA_ERR_UNSUPPORTED: return "unsupported head_dim, head grouping or geometry";
+        case BCA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case BCA_ERR_CUDA: return "CUDA runtime error";
+        case BCA_ERR_DEVICE_TIMEOUT: return "a device-side wait timed out";
+        case BCA_ERR_HOST_ONLY_PLAN: return "plan was built host-only (BCA_PLAN_HOST_ONLY)";
+        case BCA_ERR_NO_MEMORY: return "out of memory";
+        default: return "unknown error";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,645 @@
+// Forward pass of block-causal GQA attention on sm_100a.
+//
+//   kv_image_kernel : QK-Norm + 3D RoPE of the new keys (cache keys are copied as
+//                     given) and re-layout of K-hat and V into MMA-ready tile images
+//                     in the workspace, so that the attention kernel moves each K or
+//                     V tile with one bulk copy.
+//   fwd_kernel      : one CTA per work item (q-tile x two query heads of one KV
+//                     group).  Warp 0 streams K/V tiles with bulk copies (TMA engine)
+//                     into a 4-stage ring; warp 1 issues tcgen05 MMAs (S = Q K^T and
+//                     O += P V, fp32 accumulators in tensor memory); warps 4-7 and
+//                     8-11 each own one query head: they normalise, rotate and scale
+//                     their Q tile into shared memory, run the online softmax on S
+//                     rows read from tensor memory, write P (bf16) for the second MMA,
+//                     and finish with O / l and the LSE.
+//
+// The operation: attention restricted to the union of AttnSlices, with QK-Norm and
+// 3D RoPE applied to Q and K and 128/8 grouped query heads (MAGI-1 research notes
+// (zhao9797.github.io), "Autoregressive denoising DiT" and "Infra > MagiAttention >
+// Flex-Flash-Attention").  Those pages build the kernel on FlashAttention-3 for
+// Hopper; here the same online-softmax algorithm is mapped onto tcgen05 + TMEM.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.hpp"
+#include "sm100.cuh"
+
+namespace bca {
+
+using namespace sm100;
+
+namespace {
+
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait; a healthy wait is microseconds
+
+template <int D>
+struct Geo {
+    static constexpr int DPAD = (D + 15) / 16 * 16;     // MMA k-granule for bf16 is 16
+    static constexpr int PAIRS = (D / 2) / 3;           // RoPE pairs per axis
+    static constexpr int TILE_BYTES = 128 * DPAD * 2;   // one K-hat or V tile image
+};
+
+struct KVArgs {
+    const __nv_bfloat16 *k, *v, *kc, *vc;
+    const float *k_gain;
+    const uint32_t *pos;
+    const float *rope;
+    int32_t axis_off0, axis_off1, axis_off2;
+    int64_t nc, nk, nkt;
+    int hkv;
+    float eps;
+    __half *kimg;
+    __nv_bfloat16 *vimg;
+};
+
+struct FwdArgs {
+    const __nv_bfloat16 *q;
+    const float *q_gain;
+    const uint32_t *pos;
+    const float *rope;
+    int32_t axis_off0, axis_off1, axis_off2;
+    const __half *kimg;
+    const __nv_bfloat16 *vimg;
+    const Item *items;
+    const int32_t *run_off;
+    const Run *runs;
+    const uint32_t *masks;
+    int64_t nq, nkt;
+    int hq, hkv;
+    float eps, qscale;  // qscale = log2(e) / sqrt(D)
+    int o_fp32;
+    void *o;
+    float *lse;
+    int *status;
+};
+
+// ------------------------------------------------------------------ prologue math
+
+// RMS QK-Norm with gain, 3D RoPE at the packed position, then a scale; in place.
+template <int D>
+__device__ __forceinline__ void qk_prologue(float (&x)[D], uint32_t pos, const float *gain, const float *rope,
+                                            int32_t off0, int32_t off1, int32_t off2, float eps, float scale) {
+    constexpr int P = Geo<D>::PAIRS;
+    float ss = 0.f;
+#pragma unroll
+    for (int d = 0; d < D; ++d) ss = fmaf(x[d], x[d], ss);
+    const float r = rsqrtf(ss * (1.0f / D) + eps);
+#pragma unroll
+    for (int d = 0; d < D; ++d) x[d] = x[d] * r * (gain ? __ldg(gain + d) : 1.0f);
+    const int32_t p[3] = {(int32_t)(pos >> 16), (int32_t)((pos >> 8) & 255u), (int32_t)(pos & 255u)};
+    const int32_t off[3] = {off0, off1, off2};
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+        const float2 *tab = reinterpret_cast<const float2 *>(rope) + (size_t)(off[a] + p[a]) * P;
+#pragma unroll
+        for (int k = 0; k < P; ++k) {
+            const float2 cs = __ldg(tab + k);
+            const int c0 = 2 * P * a + 2 * k;
+            const float y0 = x[c0], y1 = x[c0 + 1];
+            x[c0] = y0 * cs.x - y1 * cs.y;
+            x[c0 + 1] = y0 * cs.y + y1 * cs.x;
+        }
+    }
+#pragma unroll
+    for (int d = 0; d < D; ++d) x[d] *= scale;
+}
+
+template <int D>
+__device__ __forceinline__ void load_row_bf16(const __nv_bfloat16 *src, float (&x)[D]) {
+    const uint4 *s = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+        uint4 u = __ldg(s + c);
+        const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float2 f = __bfloat1622float2(b[e]);
+            x[c * 8 + 2 * e] = f.x;
+            x[c * 8 + 2 * e + 1] = f.y;
+        }
+    }
+}
+
+// Pack values [8c, 8c+8) of x (zero past D) into one 16-byte chunk of fp16.
+template <int D>
+__device__ __forceinline__ uint4 pack_chunk_f16(const float (&x)[D], int c) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int d0 = c * 8 + 2 * e;
+        const float lo = d0 < D ? x[d0] : 0.f;
+        const float hi = d0 + 1 < D ? x[d0 + 1] : 0.f;
+        w[e] = pack_f16x2(lo, hi);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// ------------------------------------------------------------------ K-hat / V images
+
+// Tile image layout (128 x DPAD 16-bit values per (KV head, k-tile)), made of 8x8
+// core matrices of 128 contiguous bytes.  K-hat is stored as fp16: it is RMS-
+// normalised (|x| <= sqrt(D) * max|gain|), so fp16's range suffices and its 11-bit
+// significand keeps the scores 8x more precise than bf16 would; V stays bf16.
+//   K-hat: core (key group kg, d group kc) at ((kc * 16 + kg) * 64) elements,
+//          element (key, d) at + (key % 8) * 8 + d % 8.          [K-major B of S=QK^T]
+//   V    : core (d group dg, key group kc) at ((kc * DPAD/8 + dg) * 64) elements,
+//          element (d, key) at + (d % 8) * 8 + key % 8.          [K-major B of O=PV]
+template <int D>
+__global__ void __launch_bounds__(128) kv_image_kernel(KVArgs a) {
+    constexpr int DPAD = Geo<D>::DPAD;
+    __shared__ __nv_bfloat16 sv[128][DPAD + 8];
+    const int t = threadIdx.x;
+    const int64_t kt = blockIdx.x;
+    const int g = blockIdx.y;
+    const int64_t key = kt * 128 + t;
+    const size_t tile = ((size_t)g * a.nkt + kt) * (128 * DPAD);
+
+    float x[D];
+    if (key < a.nc) {
+        load_row_bf16<D>(a.kc + ((size_t)key * a.hkv + g) * D, x);
+    } else if (key < a.nk) {
+        const int64_t n = key - a.nc;
+        load_row_bf16<D>(a.k + ((size_t)n * a.hkv + g) * D, x);
+        qk_prologue<D>(x, __ldg(a.pos + n), a.k_gain, a.rope, a.axis_off0, a.axis_off1, a.axis_off2, a.eps,
+                       1.0f);
+    } else {
+#pragma unroll
+        for (int d = 0; d < D; ++d) x[d] = 0.f;
+    }
+    uint4 *kout = reinterpret_cast<uint4 *>(a.kimg + tile);
+#pragma unroll
+    for (int c = 0; c < DPAD / 8; ++c) kout[(c * 16 + t / 8) * 8 + (t % 8)] = pack_chunk_f16<D>(x, c);
+
+    // V: stage the row, then write the transposed core-matrix image
+    if (key < a.nc) {
+        load_row_bf16<D>(a.vc + ((size_t)key * a.hkv + g) * D, x);
+    } else if (key < a.nk) {
+        load_row_bf16<D>(a.v + ((size_t)(key - a.nc) * a.hkv + g) * D, x);
+    } else {
+#pragma unroll
+        for (int d = 0; d < D; ++d) x[d] = 0.f;
+    }
+#pragma unroll
+    for (int d = 0; d < DPAD; ++d) sv[t][d] = __float2bfloat16_rn(d < D ? x[d] : 0.f);
+    __syncthreads();
+    uint4 *vout = reinterpret_cast<uint4 *>(a.vimg + tile);
+#pragma unroll
+    for (int i = 0; i < DPAD / 8; ++i) {
+        const int c = t + 128 * i;  // chunk index = (kc * DPAD/8 + dg) * 8 + dd
+        const int dd = c % 8, dg = (c / 8) % (DPAD / 8), kc = c / DPAD;
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 b;
+            b.x = sv[kc * 8 + 2 * e][dg * 8 + dd];
+            b.y = sv[kc * 8 + 2 * e + 1][dg * 8 + dd];
+            w[e] = *reinterpret_cast<uint32_t *>(&b);
+        }
+        vout[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+// ------------------------------------------------------------------ attention kernel
+
+template <int D>
+struct FwdSmem {
+    static constexpr int DPAD = Geo<D>::DPAD;
+    static constexpr int STAGES = 4;
+    static constexpr int Q_BYTES = 128 * DPAD * 2;
+    static constexpr int P_BYTES = 128 * 128 * 2;
+    static constexpr int TILE = Geo<D>::TILE_BYTES;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_P = OFF_Q + 2 * Q_BYTES;
+    static constexpr int OFF_K = OFF_P + 2 * P_BYTES;
+    static constexpr int OFF_V = OFF_K + STAGES * TILE;
+    static constexpr int OFF_BAR = OFF_V + STAGES * TILE;
+    // barriers
+    static constexpr int B_KV_FULL = 0;
+    static constexpr int B_KV_EMPTY = STAGES;
+    static constexpr int B_S_FULL = 2 * STAGES;      // [2]
+    static constexpr int B_S_FREE = B_S_FULL + 2;    // [2]
+    static constexpr int B_P_FULL = B_S_FREE + 2;    // [2]
+    static constexpr int B_O_DONE = B_P_FULL + 2;    // [2]
+    static constexpr int B_Q_READY = B_O_DONE + 2;   // [2]
+    static constexpr int B_MMA_DONE = B_Q_READY + 2;
+    static constexpr int NBAR = B_MMA_DONE + 1;
+    static constexpr int OFF_TMEM_PTR = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_ABORT = OFF_TMEM_PTR + 4;
+    static constexpr int BYTES = OFF_ABORT + 12;
+    // tensor memory columns
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t COL_S = 0;    // + 128 * slot
+    static constexpr uint32_t COL_O = 256;  // + 64 * slot
+};
+
+struct RunCursor {
+    const Run *r;
+    const Run *end;
+    int32_t kt;
+    __device__ __forceinline__ RunCursor(const Run *b, const Run *e) : r(b), end(e), kt(b < e ? b->kt_begin : 0) {}
+    __device__ __forceinline__ bool valid() const { return r < end; }
+    __device__ __forceinline__ void next() {
+        if (++kt >= r->kt_end) {
+            ++r;
+            if (r < end) kt = r->kt_begin;
+        }
+    }
+};
+
+__device__ __forceinline__ void record_timeout(int *status, volatile int *abort_flag) {
+    atomicOr(status, kStatusTimeout);
+    *abort_flag = 1;
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, int *status, volatile int *abort_flag) {
+    if (*abort_flag) return false;
+    if (mbar_wait(bar, parity, kWaitTimeoutNs)) return true;
+    record_timeout(status, abort_flag);
+    return false;
+}
+
+// Same, with the outcome made uniform across the warp (for warps that go on to
+// issue warp-collective tcgen05 loads/stores).
+__device__ __forceinline__ bool warp_wait_or_abort(uint32_t bar, uint32_t parity, int *status,
+                                                   volatile int *abort_flag) {
+    const bool ok = wait_or_abort(bar, parity, status, abort_flag);
+    return __all_sync(0xffffffffu, ok);
+}
+
+template <int D>
+__global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
+    using L = FwdSmem<D>;
+    constexpr int DPAD = L::DPAD;
+    constexpr int STAGES = L::STAGES;
+    constexpr uint32_t IDESC_S = idesc_f32acc(128, 128, kFmtF16);
+    constexpr uint32_t IDESC_PV = idesc_f32acc(128, DPAD, kFmtBF16);
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + L::OFF_BAR;
+    auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::OFF_ABORT);
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + L::OFF_TMEM_PTR);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const Item item = a.items[blockIdx.x];
+    const int64_t qt = item.q_tile;
+    const int G = a.hq / a.hkv;
+    const int h0 = 2 * item.head_pair;
+    const int g = h0 / G;
+    const Run *rb = a.runs + a.run_off[qt];
+    const Run *re = a.runs + a.run_off[qt + 1];
+    int n = 0;
+    for (const Run *r = rb; r < re; ++r) n += r->kt_end - r->kt_begin;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(bar(L::B_KV_FULL + i), 1);
+            mbar_init(bar(L::B_KV_EMPTY + i), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(L::B_S_FULL + s), 1);
+            mbar_init(bar(L::B_S_FREE + s), 128);
+            mbar_init(bar(L::B_P_FULL + s), 128);
+            mbar_init(bar(L::B_O_DONE + s), 1);
+            mbar_init(bar(L::B_Q_READY + s), 128);
+        }
+        mbar_init(bar(L::B_MMA_DONE), 1);
+        mbar_fence_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 2) {
+        tmem_alloc(smem_u32(tmem_ptr), L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_ptr;
+
+    if (warp == 0) {
+        // ------------------------------------------------ producer: K/V tiles
+        if (lane == 0 && n > 0) {
+            int issued = 0;
+            RunCursor cur(rb, re);
+            for (int j = 0; j < n; ++j, cur.next()) {
+                const int stage = j % STAGES;
+                if (j >= STAGES &&
+                    !wait_or_abort(bar(L::B_KV_EMPTY + stage), ((j / STAGES) - 1) & 1, a.status, abort_flag))
+                    break;
+                const size_t tile = ((size_t)g * a.nkt + cur.kt) * (128 * DPAD);
+                mbar_arrive_expect_tx(bar(L::B_KV_FULL + stage), 2 * L::TILE);
+                bulk_g2s(sbase + L::OFF_K + stage * L::TILE, a.kimg + tile, L::TILE, bar(L::B_KV_FULL + stage));
+                bulk_g2s(sbase + L::OFF_V + stage * L::TILE, a.vimg + tile, L::TILE, bar(L::B_KV_FULL + stage));
+                ++issued;
+            }
+            // every issued copy must have landed before the CTA may exit
+            for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+                mbar_wait(bar(L::B_KV_FULL + j % STAGES), (j / STAGES) & 1, kWaitTimeoutNs);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0 && n > 0) {
+            bool ok = wait_or_abort(bar(L::B_Q_READY + 0), 0, a.status, abort_flag) &&
+                      wait_or_abort(bar(L::B_Q_READY + 1), 0, a.status, abort_flag) &&
+                      wait_or_abort(bar(L::B_KV_FULL + 0), 0, a.status, abort_flag);
+            tc_fence_after();
+            auto issue_s = [&](int slot, int stage) {
+                const uint32_t qa = sbase + L::OFF_Q + slot * L::Q_BYTES;
+                const uint32_t kb = sbase + L::OFF_K + stage * L::TILE;
+#pragma unroll
+                for (int kk = 0; kk < DPAD / 16; ++kk) {
+                    const uint64_t ad = smem_desc(qa + kk * 4096, 2048, 128);
+                    const uint64_t bd = smem_desc(kb + kk * 4096, 2048, 128);
+                    mma_f16(tbase + L::COL_S + 128 * slot, ad, bd, IDESC_S, kk > 0);
+                }
+            };
+            auto issue_pv = [&](int slot, int stage, bool acc) {
+                const uint32_t pa = sbase + L::OFF_P + slot * L::P_BYTES;
+                const uint32_t vb = sbase + L::OFF_V + stage * L::TILE;
+                constexpr uint32_t VLBO = (DPAD / 8) * 128;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t ad = smem_desc(pa + kk * 4096, 2048, 128);
+                    const uint64_t bd = smem_desc(vb + kk * 2 * VLBO, VLBO, 128);
+                    mma_f16(tbase + L::COL_O + 64 * slot, ad, bd, IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+            if (ok) {
+                for (int s = 0; s < 2; ++s) {
+                    issue_s(s, 0);
+                    mma_commit(bar(L::B_S_FULL + s));
+                }
+                for (int j = 0; j < n && ok; ++j) {
+                    const int stage = j % STAGES;
+                    const bool more = j + 1 < n;
+                    const int nstage = (j + 1) % STAGES;
+                    if (more) {
+                        ok = wait_or_abort(bar(L::B_KV_FULL + nstage), ((j + 1) / STAGES) & 1, a.status, abort_flag);
+                        tc_fence_after();
+                    }
+                    for (int s = 0; s < 2 && ok; ++s) {
+                        if (more) {
+                            ok = wait_or_abort(bar(L::B_S_FREE + s), j & 1, a.status, abort_flag);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_s(s, nstage);
+                            mma_commit(bar(L::B_S_FULL + s));
+                        }
+                        ok = wait_or_abort(bar(L::B_P_FULL + s), j & 1, a.status, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(s, stage, j > 0);
+                        mma_commit(bar(L::B_O_DONE + s));
+                    }
+                    mma_commit(bar(L::B_KV_EMPTY + stage));
+                }
+            }
+            // all issued MMAs must be complete before TMEM is released
+            mma_commit(bar(L::B_MMA_DONE));
+            mbar_wait(bar(L::B_MMA_DONE), 0, kWaitTimeoutNs);
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ------------------------------------------------ softmax / prologue / epilogue
+        const int slot = (warp - 4) / 4;
+        const int quarter = warp % 4;  // TMEM lane quarter this warp may access
+        const int row = quarter * 32 + lane;
+        const int h = h0 + slot;
+        const int64_t qrow = qt * 128 + row;
+        const bool live = qrow < a.nq;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+
+        {   // Q prologue into shared memory (fp16, core-matrix layout, K-major A operand)
+            float x[D];
+            if (live) {
+                load_row_bf16<D>(a.q + ((size_t)qrow * a.hq + h) * D, x);
+                qk_prologue<D>(x, __ldg(a.pos + qrow), a.q_gain, a.rope, a.axis_off0, a.axis_off1, a.axis_off2,
+                               a.eps, a.qscale);
+            } else {
+#pragma unroll
+                for (int d = 0; d < D; ++d) x[d] = 0.f;
+            }
+            uint4 *qs = reinterpret_cast<uint4 *>(smem + L::OFF_Q + slot * L::Q_BYTES);
+#pragma unroll
+            for (int c = 0; c < DPAD / 8; ++c) qs[(c * 16 + row / 8) * 8 + row % 8] = pack_chunk_f16<D>(x, c);
+            fence_proxy_async_smem();
+            mbar_arrive(bar(L::B_Q_READY + slot));
+        }
+
+        const uint32_t tS = tbase + lane_off + L::COL_S + 128 * slot;
+        const uint32_t tO = tbase + lane_off + L::COL_O + 64 * slot;
+        uint4 *ps = reinterpret_cast<uint4 *>(smem + L::OFF_P + slot * L::P_BYTES);
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        RunCursor cur(rb, re);
+        for (int j = 0; j < n; ++j, cur.next()) {
+            ok = warp_wait_or_abort(bar(L::B_S_FULL + slot), j & 1, a.status, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            float s[128];
+            {
+                uint32_t r[128];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 128; ++e) s[e] = __uint_as_float(r[e]);
+            }
+            tc_fence_before();
+            mbar_arrive(bar(L::B_S_FREE + slot));
+
+            if (cur.r->mask_idx >= 0) {
+                const uint4 mw = reinterpret_cast<const uint4 *>(a.masks)[(size_t)cur.r->mask_idx * 128 + row];
+                const uint32_t w4[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (!((w4[c / 32] >> (c % 32)) & 1u)) s[c] = -INFINITY;
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+            float alpha = 1.f;
+            bool rescale = false;
+            if (mx > m_ref + 8.0f) {  // lazy rescaling: move the reference only when it grows by > 2^8
+                alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - mx);
+                rescale = j > 0;
+                m_ref = mx;
+            }
+            const float msub = (m_ref == -INFINITY) ? 0.f : m_ref;
+            float sum = 0.f;
+#pragma unroll
+            for (int c = 0; c < 128; ++c) {
+                s[c] = ex2(s[c] - msub);
+                sum += s[c];
+            }
+            l = l * alpha + sum;
+
+            if (j > 0) {
+                ok = warp_wait_or_abort(bar(L::B_O_DONE + slot), (j - 1) & 1, a.status, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, rescale)) {
+                    const float f = rescale ? alpha : 1.f;
+#pragma unroll
+                    for (int c = 0; c < DPAD / 16; ++c) {
+                        uint32_t o16[16];
+                        tmem_ld16(tO + 16 * c, o16);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) o16[e] = __float_as_uint(__uint_as_float(o16[e]) * f);
+                        tmem_st16(tO + 16 * c, o16);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // P (bf16) in the core-matrix layout of the K-major A operand
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const uint4 u = make_uint4(pack_bf16x2(s[8 * c + 0], s[8 * c + 1]), pack_bf16x2(s[8 * c + 2], s[8 * c + 3]),
+                                           pack_bf16x2(s[8 * c + 4], s[8 * c + 5]), pack_bf16x2(s[8 * c + 6], s[8 * c + 7]));
+                ps[(c * 16 + row / 8) * 8 + row % 8] = u;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(L::B_P_FULL + slot));
+        }
+
+        // epilogue: O / l and LSE
+        float o[DPAD];
+#pragma unroll
+        for (int d = 0; d < DPAD; ++d) o[d] = 0.f;
+        if (n > 0 && ok) {
+            ok = warp_wait_or_abort(bar(L::B_O_DONE + slot), (n - 1) & 1, a.status, abort_flag);
+            tc_fence_after();
+            if (ok) {
+#pragma unroll
+                for (int c = 0; c < DPAD / 16; ++c) {
+                    uint32_t o16[16];
+                    tmem_ld16(tO + 16 * c, o16);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[16 * c + e] = __uint_as_float(o16[e]);
+                }
+            }
+        }
+        if (live) {
+            const bool any = l > 0.f;
+            const float inv = any ? 1.0f / l : 0.f;
+            if (a.o_fp32) {
+                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.o) + ((size_t)qrow * a.hq + h) * D);
+#pragma unroll
+                for (int c = 0; c < D / 4; ++c)
+                    dst[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv, o[4 * c + 3] * inv);
+            } else {
+                uint4 *dst =
+                    reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.o) + ((size_t)qrow * a.hq + h) * D);
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c)
+                    dst[c] = make_uint4(pack_bf16x2(o[8 * c] * inv, o[8 * c + 1] * inv),
+                                        pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
+                                        pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv),
+                                        pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
+            }
+            a.lse[(size_t)h * a.nq + qrow] = any ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tbase, L::TMEM_COLS);
+    }
+}
+
+template <int D>
+int launch_fwd_d(Plan &P, const FwdIO &io, cudaStream_t stream) {
+    using L = FwdSmem<D>;
+    const size_t img = kv_image_bytes(P);
+    auto *kimg = static_cast<__half *>(io.workspace);
+    auto *vimg = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(io.workspace) + img);
+
+    KVArgs ka;
+    ka.k = static_cast<const __nv_bfloat16 *>(io.k);
+    ka.v = static_cast<const __nv_bfloat16 *>(io.v);
+    ka.kc = static_cast<const __nv_bfloat16 *>(io.k_cache);
+    ka.vc = static_cast<const __nv_bfloat16 *>(io.v_cache);
+    ka.k_gain = io.k_gain;
+    ka.pos = P.d_pos;
+    ka.rope = P.d_rope;
+    ka.axis_off0 = P.rope_axis_off[0];
+    ka.axis_off1 = P.rope_axis_off[1];
+    ka.axis_off2 = P.rope_axis_off[2];
+    ka.nc = P.nc;
+    ka.nk = P.nk;
+    ka.nkt = P.nkt;
+    ka.hkv = P.hkv;
+    ka.eps = P.eps;
+    ka.kimg = kimg;
+    ka.vimg = vimg;
+    {
+        ProfScope ps(P, BCA_KERNEL_KV_IMAGE, stream);
+        kv_image_kernel<D><<<dim3((unsigned)P.nkt, (unsigned)P.hkv), 128, 0, stream>>>(ka);
+    }
+    if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
+
+    FwdArgs fa;
+    fa.q = static_cast<const __nv_bfloat16 *>(io.q);
+    fa.q_gain = io.q_gain;
+    fa.pos = P.d_pos;
+    fa.rope = P.d_rope;
+    fa.axis_off0 = P.rope_axis_off[0];
+    fa.axis_off1 = P.rope_axis_off[1];
+    fa.axis_off2 = P.rope_axis_off[2];
+    fa.kimg = kimg;
+    fa.vimg = vimg;
+    fa.items = P.d_items;
+    fa.run_off = P.d_run_off;
+    fa.runs = P.d_runs;
+    fa.masks = P.d_masks;
+    fa.nq = P.nq;
+    fa.nkt = P.nkt;
+    fa.hq = P.hq;
+    fa.hkv = P.hkv;
+    fa.eps = P.eps;
+    fa.qscale = 1.4426950408889634f / sqrtf((float)D);
+    fa.o_fp32 = (P.flags & BCA_O_FP32) ? 1 : 0;
+    fa.o = io.o;
+    fa.lse = io.lse;
+    fa.status = P.d_status;
+    if (cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES) != cudaSuccess)
+        return BCA_ERR_CUDA;
+    {
+        ProfScope ps(P, BCA_KERNEL_FWD, stream);
+        fwd_kernel<D><<<(unsigned)P.items.size(), 384, L::BYTES, stream>>>(fa);
+    }
+    if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
+    return BCA_OK;
+}
+
+}  // namespace
+
+size_t kv_image_bytes(const Plan &P) {
+    const size_t b = (size_t)P.hkv * (size_t)P.nkt * 128 * (size_t)P.dpad * 2;
+    return (b + 255) / 256 * 256;
+}
+
+size_t fwd_workspace_bytes(const Plan &P) { return 2 * kv_image_bytes(P); }
+
+int launch_fwd(Plan &P, const FwdIO &io, cudaStream_t stream) {
+    if (P.nq == 0) return BCA_OK;
+    switch (P.d) {
+        case 24: return launch_fwd_d<24>(P, io, stream);
+        case 32: return launch_fwd_d<32>(P, io, stream);
+        case 48: return launch_fwd_d<48>(P, io, stream);
+        default: return BCA_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace bca

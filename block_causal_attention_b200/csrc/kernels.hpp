@@ -1,0 +1,38 @@
+// Launch interface between the C ABI (api.cpp) and the CUDA kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "plan.hpp"
+
+namespace bca {
+
+// status-word bits written by kernels
+constexpr int kStatusTimeout = 0x1;
+
+struct FwdIO {
+    const void *q, *k, *v, *k_cache, *v_cache;
+    const float *q_gain, *k_gain;
+    void *o;
+    float *lse;
+    void *workspace;
+};
+
+// Bytes of each K-hat / V image (all KV heads, all k-tiles), 256-byte rounded.
+size_t kv_image_bytes(const Plan &plan);
+size_t fwd_workspace_bytes(const Plan &plan);
+
+// Bracket a launch with events when the plan is profiling (no-op otherwise).
+struct ProfScope {
+    Plan &plan;
+    int kernel;
+    cudaStream_t stream;
+    cudaEvent_t start = nullptr;
+    ProfScope(Plan &p, int k, cudaStream_t s);
+    ~ProfScope();
+};
+
+// Enqueue the forward on `stream`.  Returns BCA_OK or BCA_ERR_CUDA.
+int launch_fwd(Plan &plan, const FwdIO &io, cudaStream_t stream);
+
+}  // namespace bca

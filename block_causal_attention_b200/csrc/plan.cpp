@@ -1,0 +1,306 @@
+// Mask compiler: AttnSlices -> per-(128 x 128) tile classes -> runs -> work items.
+//
+// The mask is the union of the slices (MAGI-1 research notes (zhao9797.github.io),
+// "Infra > MagiAttention > Flex-Flash-Attention": masks are compositions of
+// (QRange, KRange, MaskType) slices; interview with Zhang Zheng (zhengguannews),
+// the q_range / k_range answer).  Work items are ordered by the visible area of
+// their q-tile, largest first, which is the pages' "balance the unmasked area"
+// cost model (interview, the dispatch-solver answer; research notes, "Dispatch
+// solver") applied to the SMs of one GPU instead of CP ranks.
+#include "plan.hpp"
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <thread>
+
+namespace bca {
+
+namespace {
+
+struct Interval {
+    int64_t a, b;  // [a, b)
+};
+
+// Visible keys of row i through slice s, as one interval (may be empty).
+inline Interval slice_row_interval(const bca_slice &s, int64_t i) {
+    if (s.type == BCA_SLICE_FULL) return {s.k_begin, s.k_end};
+    // causal, bottom-right aligned: j - k0 <= (i - q0) + (|k| - |q|)
+    int64_t lim = s.k_begin + (i - s.q_begin) + ((s.k_end - s.k_begin) - (s.q_end - s.q_begin)) + 1;
+    return {s.k_begin, std::min(s.k_end, std::max(lim, s.k_begin))};
+}
+
+// Per-q-tile compile output, merged in q-tile order afterwards.
+struct TileOut {
+    std::vector<Run> runs;          // mask_idx local to this q-tile
+    std::vector<uint32_t> masks;    // local partial masks
+    int64_t pairs = 0, nfull = 0, npartial = 0;
+    int32_t ntiles = 0;
+};
+
+void compile_q_tile(const Plan &P, int64_t qt, TileOut &out) {
+    const int64_t r0 = qt * kTileQ;
+    const int nr = (int)std::min<int64_t>(kTileQ, P.nq - r0);
+    // 1. merged visible intervals of every row
+    std::vector<std::vector<Interval>> iv(nr);
+    for (const bca_slice &s : P.slices) {
+        int64_t lo = std::max(s.q_begin, r0), hi = std::min(s.q_end, r0 + nr);
+        for (int64_t i = lo; i < hi; ++i) {
+            Interval x = slice_row_interval(s, i);
+            if (x.b > x.a) iv[i - r0].push_back(x);
+        }
+    }
+    int64_t tmin = INT64_MAX, tmax = -1;
+    for (auto &v : iv) {
+        if (v.empty()) continue;
+        std::sort(v.begin(), v.end(), [](const Interval &x, const Interval &y) { return x.a < y.a; });
+        std::vector<Interval> m;
+        for (const Interval &x : v) {
+            if (!m.empty() && x.a <= m.back().b) m.back().b = std::max(m.back().b, x.b);
+            else m.push_back(x);
+        }
+        v.swap(m);
+        for (const Interval &x : v) {
+            out.pairs += x.b - x.a;
+            tmin = std::min(tmin, x.a / kTileK);
+            tmax = std::max(tmax, (x.b - 1) / kTileK);
+        }
+    }
+    if (tmax < 0) return;
+    // 2. per k-tile: rows that cover it fully (difference array) and rows that
+    //    cover it partly
+    const int64_t span = tmax - tmin + 1;
+    std::vector<int32_t> diff(span + 1, 0);
+    std::vector<uint8_t> touched(span, 0);
+    for (const auto &v : iv) {
+        for (const Interval &x : v) {
+            int64_t fa = (x.a + kTileK - 1) / kTileK, fb = x.b / kTileK;  // fully covered [fa, fb)
+            if (fa < fb) {
+                diff[fa - tmin] += 1;
+                diff[fb - tmin] -= 1;
+            }
+            int64_t ta = x.a / kTileK, tb = (x.b - 1) / kTileK;
+            if (!(fa <= ta && ta < fb)) touched[ta - tmin] = 1;
+            if (!(fa <= tb && tb < fb)) touched[tb - tmin] = 1;
+        }
+    }
+    // 3. classify and emit runs
+    int32_t cnt = 0;
+    for (int64_t t = tmin; t <= tmax; ++t) {
+        cnt += diff[t - tmin];
+        const bool in_range = (t + 1) * kTileK <= P.nk;
+        const bool tch = touched[t - tmin] != 0;
+        if (cnt == nr && !tch && in_range) {
+            if (!out.runs.empty() && out.runs.back().mask_idx < 0 && out.runs.back().kt_end == t)
+                out.runs.back().kt_end = (int32_t)(t + 1);
+            else
+                out.runs.push_back({(int32_t)t, (int32_t)(t + 1), -1, 0});
+            out.nfull++;
+            out.ntiles++;
+        } else if (cnt == 0 && !tch) {
+            continue;  // empty
+        } else {
+            const int32_t idx = (int32_t)(out.masks.size() / (kTileQ * 4));
+            out.masks.resize(out.masks.size() + kTileQ * 4, 0u);
+            uint32_t *mk = out.masks.data() + (size_t)idx * kTileQ * 4;
+            const int64_t k0 = t * kTileK, k1 = k0 + kTileK;
+            for (int r = 0; r < nr; ++r) {
+                for (const Interval &x : iv[r]) {
+                    int64_t a = std::max(x.a, k0), b = std::min(x.b, k1);
+                    for (int64_t j = a; j < b; ++j) mk[r * 4 + (j - k0) / 32] |= 1u << ((j - k0) % 32);
+                }
+            }
+            out.runs.push_back({(int32_t)t, (int32_t)(t + 1), idx, 0});
+            out.npartial++;
+            out.ntiles++;
+        }
+    }
+}
+
+}  // namespace
+
+int validate_problem(const bca_problem *p, Plan &P) {
+    if (!p) return BCA_ERR_INVALID_ARGUMENT;
+    if (p->flags & ~(BCA_O_FP32 | BCA_PLAN_HOST_ONLY)) return BCA_ERR_INVALID_ARGUMENT;
+    if (p->num_q_heads <= 0 || p->num_kv_heads <= 0) return BCA_ERR_INVALID_ARGUMENT;
+    if (p->num_q_heads % p->num_kv_heads != 0) return BCA_ERR_UNSUPPORTED;
+    if ((p->num_q_heads / p->num_kv_heads) % 2 != 0) return BCA_ERR_UNSUPPORTED;
+    if (p->head_dim != 24 && p->head_dim != 32 && p->head_dim != 48) return BCA_ERR_UNSUPPORTED;
+    if (p->num_videos < 0 || (p->num_videos > 0 && !p->videos)) return BCA_ERR_INVALID_ARGUMENT;
+    if (p->num_cache_keys < 0) return BCA_ERR_INVALID_ARGUMENT;
+    if (p->num_slices < 0 || (p->num_slices > 0 && !p->slices)) return BCA_ERR_INVALID_ARGUMENT;
+    for (int a = 0; a < 3; ++a)
+        if (!(p->rope_base[a] > 0.0f) || !std::isfinite(p->rope_base[a])) return BCA_ERR_INVALID_ARGUMENT;
+    if (!(p->norm_eps >= 0.0f) || !std::isfinite(p->norm_eps)) return BCA_ERR_INVALID_ARGUMENT;
+
+    P.hq = p->num_q_heads;
+    P.hkv = p->num_kv_heads;
+    P.d = p->head_dim;
+    P.dpad = (p->head_dim + 15) / 16 * 16;
+    P.flags = p->flags;
+    P.eps = p->norm_eps;
+    for (int a = 0; a < 3; ++a) P.base[a] = p->rope_base[a];
+    P.nc = p->num_cache_keys;
+    int64_t nq = 0;
+    P.videos.assign(p->videos, p->videos + p->num_videos);
+    for (const bca_video &v : P.videos) {
+        if (v.num_chunks < 0 || v.frames <= 0 || v.height <= 0 || v.width <= 0 || v.t0 < 0)
+            return BCA_ERR_INVALID_ARGUMENT;
+        // packed RoPE positions: t < 65536, h, w < 256
+        if (v.height > 256 || v.width > 256) return BCA_ERR_UNSUPPORTED;
+        if ((int64_t)v.t0 + (int64_t)v.num_chunks * v.frames > 65536) return BCA_ERR_UNSUPPORTED;
+        nq += (int64_t)v.num_chunks * v.frames * v.height * v.width;
+    }
+    P.nq = nq;
+    P.nk = P.nc + nq;
+    if (P.nq >= ((int64_t)1 << 31) || P.nk >= ((int64_t)1 << 31)) return BCA_ERR_UNSUPPORTED;
+
+    if (p->slices) {
+        P.slices.assign(p->slices, p->slices + p->num_slices);
+        for (const bca_slice &s : P.slices) {
+            if (s.type != BCA_SLICE_FULL && s.type != BCA_SLICE_CAUSAL) return BCA_ERR_BAD_SLICE;
+            if (s.q_begin < 0 || s.q_begin > s.q_end || s.q_end > P.nq) return BCA_ERR_BAD_SLICE;
+            if (s.k_begin < 0 || s.k_begin > s.k_end || s.k_end > P.nk) return BCA_ERR_BAD_SLICE;
+        }
+    } else {
+        // default: block-causal per video; the cache is visible to the first video
+        int64_t qoff = 0;
+        for (size_t vi = 0; vi < P.videos.size(); ++vi) {
+            const bca_video &v = P.videos[vi];
+            const int64_t C = (int64_t)v.frames * v.height * v.width;
+            const int64_t kbase = P.nc + qoff;
+            for (int c = 0; c < v.num_chunks; ++c) {
+                bca_slice s;
+                s.q_begin = qoff + c * C;
+                s.q_end = qoff + (c + 1) * C;
+                s.k_begin = (vi == 0) ? 0 : kbase;
+                s.k_end = kbase + (c + 1) * C;
+                s.type = BCA_SLICE_FULL;
+                P.slices.push_back(s);
+            }
+            qoff += (int64_t)v.num_chunks * C;
+        }
+    }
+    return BCA_OK;
+}
+
+int compile_plan(Plan &P) {
+    P.nqt = (P.nq + kTileQ - 1) / kTileQ;
+    P.nkt = (P.nk + kTileK - 1) / kTileK;
+
+    // ---- mask compile, parallel over q-tiles (static contiguous ranges) ----
+    std::vector<TileOut> outs(P.nqt);
+    unsigned nth = std::max(1u, std::min(32u, std::thread::hardware_concurrency()));
+    if (P.nqt < 64) nth = 1;
+    {
+        std::vector<std::thread> th;
+        for (unsigned t = 0; t < nth; ++t) {
+            th.emplace_back([&, t]() {
+                for (int64_t qt = t; qt < P.nqt; qt += nth) compile_q_tile(P, qt, outs[qt]);
+            });
+        }
+        for (auto &x : th) x.join();
+    }
+    P.run_off.assign(P.nqt + 1, 0);
+    P.qt_tiles.assign(P.nqt, 0);
+    P.runs.clear();
+    P.masks.clear();
+    P.visible_pairs = P.nfull = P.npartial = 0;
+    for (int64_t qt = 0; qt < P.nqt; ++qt) {
+        TileOut &o = outs[qt];
+        const int32_t base = (int32_t)(P.masks.size() / (kTileQ * 4));
+        P.run_off[qt] = (int32_t)P.runs.size();
+        for (Run r : o.runs) {
+            if (r.mask_idx >= 0) r.mask_idx += base;
+            P.runs.push_back(r);
+        }
+        P.masks.insert(P.masks.end(), o.masks.begin(), o.masks.end());
+        P.qt_tiles[qt] = o.ntiles;
+        P.visible_pairs += o.pairs;
+        P.nfull += o.nfull;
+        P.npartial += o.npartial;
+        std::vector<Run>().swap(o.runs);
+        std::vector<uint32_t>().swap(o.masks);
+    }
+    P.run_off[P.nqt] = (int32_t)P.runs.size();
+
+    // ---- items, longest first; ties grouped by KV group then q-tile so that CTAs
+    //      running together stream the same K/V tiles ----
+    const int npairs = P.hq / 2, G = P.hq / P.hkv;
+    P.items.clear();
+    P.items.reserve((size_t)P.nqt * npairs);
+    for (int64_t qt = 0; qt < P.nqt; ++qt)
+        for (int hp = 0; hp < npairs; ++hp) P.items.push_back({(int32_t)qt, hp});
+    std::stable_sort(P.items.begin(), P.items.end(), [&](const Item &x, const Item &y) {
+        const int32_t cx = P.qt_tiles[x.q_tile], cy = P.qt_tiles[y.q_tile];
+        if (cx != cy) return cx > cy;
+        const int gx = 2 * x.head_pair / G, gy = 2 * y.head_pair / G;
+        if (gx != gy) return gx < gy;
+        if (x.q_tile != y.q_tile) return x.q_tile < y.q_tile;
+        return x.head_pair < y.head_pair;
+    });
+
+    // ---- positions and RoPE tables ----
+    P.pos.resize(P.nq);
+    int32_t tmax = 0, hmax = 0, wmax = 0;
+    int64_t n = 0;
+    for (const bca_video &v : P.videos) {
+        for (int c = 0; c < v.num_chunks; ++c)
+            for (int f = 0; f < v.frames; ++f)
+                for (int y = 0; y < v.height; ++y)
+                    for (int x = 0; x < v.width; ++x) {
+                        const uint32_t t = (uint32_t)(v.t0 + c * v.frames + f);
+                        P.pos[n++] = (t << 16) | ((uint32_t)y << 8) | (uint32_t)x;
+                        tmax = std::max<int32_t>(tmax, (int32_t)t);
+                        hmax = std::max(hmax, y);
+                        wmax = std::max(wmax, x);
+                    }
+    }
+    const int pairs = (P.d / 2) / 3;
+    P.rope_pairs = pairs;
+    const int32_t ext[3] = {tmax + 1, hmax + 1, wmax + 1};
+    P.rope_axis_off[0] = 0;
+    P.rope_axis_off[1] = ext[0];
+    P.rope_axis_off[2] = ext[0] + ext[1];
+    P.rope.assign((size_t)(ext[0] + ext[1] + ext[2]) * pairs * 2, 0.0f);
+    for (int a = 0; a < 3; ++a) {
+        for (int32_t pp = 0; pp < ext[a]; ++pp) {
+            for (int k = 0; k < pairs; ++k) {
+                const double ang = (double)pp * std::pow((double)P.base[a], -(double)k / (double)pairs);
+                const size_t at = ((size_t)(P.rope_axis_off[a] + pp) * pairs + k) * 2;
+                P.rope[at] = (float)std::cos(ang);
+                P.rope[at + 1] = (float)std::sin(ang);
+            }
+        }
+    }
+    return BCA_OK;
+}
+
+int expand_rows(const Plan &P, int64_t r0, int64_t r1, uint8_t *out) {
+    if (r0 < 0 || r1 < r0 || r1 > P.nq || !out) return BCA_ERR_INVALID_ARGUMENT;
+    std::memset(out, 0, (size_t)(r1 - r0) * (size_t)P.nk);
+    for (int64_t i = r0; i < r1; ++i) {
+        const int64_t qt = i / kTileQ;
+        const int r = (int)(i - qt * kTileQ);
+        uint8_t *row = out + (size_t)(i - r0) * (size_t)P.nk;
+        for (int32_t ri = P.run_off[qt]; ri < P.run_off[qt + 1]; ++ri) {
+            const Run &run = P.runs[ri];
+            for (int32_t t = run.kt_begin; t < run.kt_end; ++t) {
+                const int64_t k0 = (int64_t)t * kTileK;
+                for (int j = 0; j < kTileK; ++j) {
+                    const int64_t key = k0 + j;
+                    bool vis;
+                    if (run.mask_idx < 0) vis = true;
+                    else vis = (P.masks[((size_t)run.mask_idx * kTileQ + r) * 4 + j / 32] >> (j % 32)) & 1u;
+                    if (vis) {
+                        if (key >= P.nk) return BCA_ERR_BAD_SLICE;  // a compiled key out of range
+                        row[key] = (uint8_t)(row[key] + 1);
+                    }
+                }
+            }
+        }
+    }
+    return BCA_OK;
+}
+
+}  // namespace bca

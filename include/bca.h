@@ -1,0 +1,170 @@
+/*
+ * bca.h - C ABI of the block-causal attention library (libbca.so) for NVIDIA B200
+ * (sm_100a).  Plain pointers and sizes only; no C++ or framework types cross it.
+ *
+ * The operation (all citations name the MAGI-1 pages by title and section):
+ *
+ *   Block-causal attention: tokens attend fully to the tokens of their own video
+ *   chunk and to every token of earlier chunks, never to later chunks
+ *   ("Magi-1 开源&刷屏" (163.com), the block-causal attention bullets; MAGI-1
+ *   research notes (zhao9797.github.io), "Model architecture > Overall pipeline").
+ *   The mask is a union of AttnSlices (q-range, k-range, full|causal), which also
+ *   expresses packed variable-length videos and KV-range limits (MAGI-1 research
+ *   notes, "Infra > MagiAttention > Flex-Flash-Attention" and "Inference tricks >
+ *   KV Cache"; interview with Zhang Zheng (zhengguannews), the q_range/k_range
+ *   answer).  Queries and keys pass through QK-Norm and a 3D (t, h, w) RoPE before
+ *   the dot product, and heads are grouped (GQA, 128 query heads over 8 KV heads)
+ *   (MAGI-1 research notes, "Autoregressive denoising DiT" and Table 2).
+ *
+ *   For query token i, query head h, KV head g = h / (Hq / Hkv):
+ *     qh_i = RoPE(pos_i, RMSNorm(q_i))   kh_j = RoPE(pos_j, RMSNorm(k_j))
+ *     s_ij = qh_i . kh_j / sqrt(D) over the keys j visible to i,
+ *     LSE_i = log sum_j exp(s_ij),  O_i = sum_j exp(s_ij - LSE_i) v_j.
+ *   A row that sees no key has O = 0 and LSE = -inf.
+ *
+ * Key index space = [cache keys | new keys]: cache key c has index c, new token n
+ * has key index num_cache_keys + n.  Cache keys are taken as already normalised
+ * and rotated (they are the features of earlier chunks) and are used as given.
+ *
+ * Layouts (token-major, contiguous, row-major):
+ *   q, dout, o, dq ........ [Nq][Hq][D]
+ *   k, v, dk, dv .......... [Nq][Hkv][D]       (new tokens)
+ *   k_cache, v_cache, dk_cache, dv_cache [Nc][Hkv][D]
+ *   lse ................... [Hq][Nq] fp32, natural log
+ *   bf16 tensors are IEEE bfloat16; every pointer must be 16-byte aligned.
+ *
+ * Ownership: the caller owns every tensor, the workspace and the stream.  A plan
+ * owns its host tables and the device metadata it uploads, freed by
+ * bca_plan_destroy.  bca_fwd and bca_bwd are asynchronous on the given stream and
+ * never allocate.
+ *
+ * Errors: every int-returning call returns BCA_OK (0) or a negative BCA_ERR_*.
+ * Argument checks happen on the host before any launch; a failed check launches
+ * nothing.  No call traps the GPU.  Device-side waits are bounded: a wait that runs
+ * out records BCA_ERR_DEVICE_TIMEOUT in the plan's status word (read it with
+ * bca_status).
+ */
+#ifndef BCA_H
+#define BCA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BCA_OK 0
+#define BCA_ERR_INVALID_ARGUMENT (-1)  /* NULL pointer, bad size, bad flag */
+#define BCA_ERR_BAD_SLICE (-2)         /* slice out of range, begin > end, bad type */
+#define BCA_ERR_UNSUPPORTED (-3)       /* head_dim / head grouping / geometry not supported */
+#define BCA_ERR_MISALIGNED (-4)        /* a pointer is not 16-byte aligned */
+#define BCA_ERR_CUDA (-5)              /* a CUDA runtime call failed */
+#define BCA_ERR_DEVICE_TIMEOUT (-6)    /* a device-side wait ran out (see bca_status) */
+#define BCA_ERR_HOST_ONLY_PLAN (-7)    /* plan was built with BCA_PLAN_HOST_ONLY */
+#define BCA_ERR_NO_MEMORY (-8)         /* host or device allocation failed in bca_plan_create */
+
+/* AttnSlice type */
+#define BCA_SLICE_FULL 0
+#define BCA_SLICE_CAUSAL 1 /* bottom-right aligned: j-k0 <= (i-q0) + (|k| - |q|) */
+
+/* bca_problem.flags */
+#define BCA_O_FP32 0x1u          /* write O as fp32 instead of bf16 */
+#define BCA_PLAN_HOST_ONLY 0x2u  /* compile the mask on the host only (no CUDA calls) */
+
+/* bca_workspace_bytes(pass) */
+#define BCA_PASS_FWD 0
+#define BCA_PASS_BWD 1
+
+/* One AttnSlice: query rows [q_begin, q_end) see keys [k_begin, k_end), fully or
+ * causally.  Same memory layout as int64 [5]. */
+typedef struct {
+    int64_t q_begin, q_end, k_begin, k_end, type;
+} bca_slice;
+
+/* Geometry of the new tokens of one video, packed in order: tokens are numbered
+ * chunk, latent frame, row, column (raster order); token (c, f, y, x) has RoPE
+ * position (t0 + c*frames + f, y, x).  Same layout as int32 [5]. */
+typedef struct {
+    int32_t num_chunks, frames, height, width, t0;
+} bca_video;
+
+typedef struct {
+    int32_t num_q_heads;        /* Hq */
+    int32_t num_kv_heads;       /* Hkv; Hq % Hkv == 0 and (Hq / Hkv) even */
+    int32_t head_dim;           /* D in {24, 32, 48} */
+    int32_t num_videos;
+    const bca_video *videos;    /* Nq = sum of chunks*frames*height*width */
+    int64_t num_cache_keys;     /* Nc */
+    int32_t num_slices;
+    const bca_slice *slices;    /* NULL => block-causal per video, cache visible to
+                                   every chunk of the first video */
+    float rope_base[3];         /* RoPE base per axis (t, h, w) */
+    float norm_eps;             /* QK-Norm epsilon */
+    uint32_t flags;             /* BCA_O_FP32 | BCA_PLAN_HOST_ONLY */
+} bca_problem;
+
+typedef struct bca_plan_s *bca_plan_t;
+
+/* Plan statistics (host introspection; used by tests and the benchmark). */
+typedef struct {
+    int64_t num_q, num_k, num_cache;
+    int64_t num_q_tiles, num_k_tiles;
+    int64_t num_runs;            /* runs of consecutive k-tiles over all q-tiles */
+    int64_t num_full_tiles, num_partial_tiles;
+    int64_t num_items;           /* forward work items (q-tile x head pair) */
+    int64_t visible_pairs;       /* visible (query, key) pairs per head */
+    int32_t head_dim_padded;     /* D rounded up to the MMA k-granule (16) */
+    int32_t tile_q, tile_k;
+} bca_plan_info;
+
+/* Compile the mask and build a plan: validates the problem, classifies every
+ * (128 x 128) tile as empty / full / partial (with a bitmask), orders the forward
+ * work items longest-first by visible area (the load-balancing idea of the pages'
+ * dispatch solver: balance mask area, MAGI-1 research notes, "Infra > MagiAttention
+ * > Dispatch solver"), and, unless BCA_PLAN_HOST_ONLY, uploads the metadata to the
+ * current device.  On success *out owns everything; on failure *out is NULL. */
+int bca_plan_create(const bca_problem *problem, bca_plan_t *out);
+void bca_plan_destroy(bca_plan_t plan);
+int bca_plan_get_info(bca_plan_t plan, bca_plan_info *info);
+
+/* Expand the compiled tiles of query rows [row_begin, row_end) back into a dense
+ * coverage map: out[(i - row_begin) * Nk + j] = number of compiled tiles that
+ * mark pair (i, j) visible (0 or 1 for a correct plan).  Host only. */
+int bca_plan_expand_rows(bca_plan_t plan, int64_t row_begin, int64_t row_end, uint8_t *out);
+
+/* Bytes of caller-provided device workspace a pass needs (16-byte aligned). */
+size_t bca_workspace_bytes(bca_plan_t plan, int pass);
+
+/* Forward.  q, k, v, k_cache, v_cache: bf16 (k_cache/v_cache NULL iff Nc == 0);
+ * q_gain, k_gain: fp32 [D] QK-Norm gains or NULL (= ones); o: bf16 or fp32
+ * (BCA_O_FP32) [Nq][Hq][D]; lse: fp32 [Hq][Nq]; workspace: bca_workspace_bytes(FWD)
+ * bytes; stream: a cudaStream_t (NULL = legacy default stream). */
+int bca_fwd(bca_plan_t plan, const void *q, const void *k, const void *v,
+            const void *k_cache, const void *v_cache, const float *q_gain,
+            const float *k_gain, void *o, float *lse, void *workspace, void *stream);
+
+/* Kernel kinds for per-kernel timing */
+#define BCA_KERNEL_KV_IMAGE 0  /* K-hat prologue + K/V tile images */
+#define BCA_KERNEL_FWD 1       /* attention forward */
+#define BCA_KERNEL_COUNT 2
+
+/* Per-kernel device timing, a tracing aid.  While enabled (enable != 0), every
+ * kernel that bca_fwd launches for this plan is bracketed by two CUDA events
+ * recorded on its stream.  bca_profile_read waits for those events and returns, for
+ * one kernel kind, the number of launches and their summed device time in ms since
+ * the last read (or enable), then forgets them.  Disabled by default. */
+int bca_profile_enable(bca_plan_t plan, int enable);
+int bca_profile_read(bca_plan_t plan, int kernel, int64_t *launches, double *total_ms);
+
+/* Device status word of the plan (timeouts recorded by its kernels).  Synchronises
+ * the stream, returns BCA_OK or the recorded error, and clears it. */
+int bca_status(bca_plan_t plan, void *stream);
+
+const char *bca_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BCA_H */

@@ -232,6 +232,16 @@ static double attend_row(const double *q, const double *kh, const double *v, int
     return lse;
 }
 
+/* Dense mask rows for a list of query rows: masks[r * nk + j]. */
+static uint8_t *mask_rows(const int64_t *sl, int ns, int64_t nk, const int64_t *rows, int64_t nr)
+{
+    uint8_t *m = (uint8_t *)malloc((size_t)(nr > 0 ? nr : 1) * (size_t)(nk > 0 ? nk : 1));
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nr; ++r)
+        orc_mask_row(sl, ns, nk, rows[r], m + (size_t)r * (size_t)nk);
+    return m;
+}
+
 /* Forward for a list of query rows, every head.
  * qh: [nr][Hq][D] = post-prologue queries of those rows (in list order);
  * kh, v: [nk][Hkv][D]; O: [nr][Hq][D]; lse: [nr][Hq] (natural log). */
@@ -242,19 +252,13 @@ void orc_fwd_rows(const double *qh, const int64_t *rows, int64_t nr,
 {
     int G = Hq / Hkv;
     double scale = 1.0 / sqrt((double)D);
-#pragma omp parallel
-    {
-        uint8_t *row = (uint8_t *)malloc((size_t)nk);
-#pragma omp for schedule(dynamic, 1)
-        for (int64_t r = 0; r < nr; ++r) {
-            orc_mask_row(sl, ns, nk, rows[r], row);
-            for (int h = 0; h < Hq; ++h)
-                lse[r * Hq + h] = attend_row(qh + ((size_t)r * Hq + h) * D, kh, v, nk, row,
-                                             Hkv, h / G, D, scale,
-                                             O + ((size_t)r * Hq + h) * D);
-        }
-        free(row);
-    }
+    uint8_t *m = mask_rows(sl, ns, nk, rows, nr);
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int64_t r = 0; r < nr; ++r)
+        for (int h = 0; h < Hq; ++h)
+            lse[r * Hq + h] = attend_row(qh + ((size_t)r * Hq + h) * D, kh, v, nk, m + (size_t)r * (size_t)nk,
+                                         Hkv, h / G, D, scale, O + ((size_t)r * Hq + h) * D);
+    free(m);
 }
 
 /* dq-hat for a list of rows: forward of the row, Di = dO_i . O_i,
@@ -268,45 +272,42 @@ void orc_bwd_rows(const double *qh, const int64_t *rows, int64_t nr,
     int G = Hq / Hkv;
     double scale = 1.0 / sqrt((double)D);
     orc_fwd_rows(qh, rows, nr, kh, v, nk, sl, ns, Hq, Hkv, D, O, lse);
-#pragma omp parallel
-    {
-        uint8_t *row = (uint8_t *)malloc((size_t)nk);
-#pragma omp for schedule(dynamic, 1)
-        for (int64_t r = 0; r < nr; ++r) {
-            orc_mask_row(sl, ns, nk, rows[r], row);
-            for (int h = 0; h < Hq; ++h) {
-                int g = h / G;
-                const double *q = qh + ((size_t)r * Hq + h) * D;
-                const double *doi = dO + ((size_t)r * Hq + h) * D;
-                const double *oi = O + ((size_t)r * Hq + h) * D;
-                double *dq = dqh + ((size_t)r * Hq + h) * D;
-                double L = lse[r * Hq + h];
-                double Di = 0.0;
-                for (int d = 0; d < D; ++d) {
-                    Di += doi[d] * oi[d];
-                    dq[d] = 0.0;
-                }
-                if (L == -INFINITY)
+    uint8_t *m = mask_rows(sl, ns, nk, rows, nr);
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int64_t r = 0; r < nr; ++r) {
+        for (int h = 0; h < Hq; ++h) {
+            const uint8_t *row = m + (size_t)r * (size_t)nk;
+            int g = h / G;
+            const double *q = qh + ((size_t)r * Hq + h) * D;
+            const double *doi = dO + ((size_t)r * Hq + h) * D;
+            const double *oi = O + ((size_t)r * Hq + h) * D;
+            double *dq = dqh + ((size_t)r * Hq + h) * D;
+            double L = lse[r * Hq + h];
+            double Di = 0.0;
+            for (int d = 0; d < D; ++d) {
+                Di += doi[d] * oi[d];
+                dq[d] = 0.0;
+            }
+            if (L == -INFINITY)
+                continue;
+            for (int64_t j = 0; j < nk; ++j) {
+                if (!row[j])
                     continue;
-                for (int64_t j = 0; j < nk; ++j) {
-                    if (!row[j])
-                        continue;
-                    const double *kj = kh + ((size_t)j * Hkv + g) * D;
-                    const double *vj = v + ((size_t)j * Hkv + g) * D;
-                    double s = 0.0, dp = 0.0;
-                    for (int d = 0; d < D; ++d) {
-                        s += q[d] * kj[d];
-                        dp += doi[d] * vj[d];
-                    }
-                    double P = exp(s * scale - L);
-                    double dS = P * (dp - Di);
-                    for (int d = 0; d < D; ++d)
-                        dq[d] += dS * kj[d] * scale;
+                const double *kj = kh + ((size_t)j * Hkv + g) * D;
+                const double *vj = v + ((size_t)j * Hkv + g) * D;
+                double s = 0.0, dp = 0.0;
+                for (int d = 0; d < D; ++d) {
+                    s += q[d] * kj[d];
+                    dp += doi[d] * vj[d];
                 }
+                double P = exp(s * scale - L);
+                double dS = P * (dp - Di);
+                for (int d = 0; d < D; ++d)
+                    dq[d] += dS * kj[d] * scale;
             }
         }
-        free(row);
     }
+    free(m);
 }
 
 /* dk-hat and dv for a list of keys, for query heads [h_begin, h_end) only (all heads
