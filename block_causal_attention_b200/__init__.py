@@ -62,6 +62,13 @@ class Plan:
                    "bca_plan_expand_rows")
         return out
 
+    def expand_cols(self, k0: int, k1: int) -> np.ndarray:
+        """Coverage of keys [k0, k1) from the backward's transposed tables: [k1-k0, Nq]."""
+        out = np.zeros((k1 - k0, self.nq), dtype=np.uint8)
+        _abi.check(self._lib.bca_plan_expand_cols(self._h, k0, k1, out.ctypes.data if out.size else None),
+                   "bca_plan_expand_cols")
+        return out
+
     def workspace_bytes(self, pass_: int = _abi.BCA_PASS_FWD) -> int:
         return int(self._lib.bca_workspace_bytes(self._h, pass_))
 

@@ -30,6 +30,7 @@ BCA_PASS_BWD = 1
 
 # every symbol include/bca.h declares
 EXPORTS = ("bca_plan_create", "bca_plan_destroy", "bca_plan_get_info", "bca_plan_expand_rows",
+           "bca_plan_expand_cols",
            "bca_workspace_bytes", "bca_fwd", "bca_profile_enable", "bca_profile_read", "bca_status",
            "bca_error_string")
 BCA_KERNEL_KV_IMAGE = 0
@@ -90,6 +91,8 @@ def lib() -> ctypes.CDLL:
         L.bca_plan_get_info.restype = i32
         L.bca_plan_expand_rows.argtypes = [vp, i64, i64, vp]
         L.bca_plan_expand_rows.restype = i32
+        L.bca_plan_expand_cols.argtypes = [vp, i64, i64, vp]
+        L.bca_plan_expand_cols.restype = i32
         L.bca_workspace_bytes.argtypes = [vp, i32]
         L.bca_workspace_bytes.restype = ctypes.c_size_t
         L.bca_fwd.argtypes = [vp] * 12

@@ -52,8 +52,12 @@ int upload(bca::Plan &P) {
     const size_t s_items = round256(std::max<size_t>(1, P.items.size()) * sizeof(Item));
     const size_t s_pos = round256(std::max<size_t>(1, P.pos.size()) * sizeof(uint32_t));
     const size_t s_rope = round256(std::max<size_t>(1, P.rope.size()) * sizeof(float));
+    const size_t s_coloff = round256(P.col_off.size() * sizeof(int32_t));
+    const size_t s_colruns = round256(std::max<size_t>(1, P.col_runs.size()) * sizeof(Run));
+    const size_t s_bitems = round256(std::max<size_t>(1, P.bwd_items.size()) * sizeof(int32_t));
     const size_t s_status = 256;
-    const size_t total = s_runoff + s_runs + s_masks + s_items + s_pos + s_rope + s_status;
+    const size_t total = s_runoff + s_runs + s_masks + s_items + s_pos + s_rope + s_coloff + s_colruns +
+                         s_bitems + s_status;
     if (cudaGetDevice(&P.device) != cudaSuccess) return BCA_ERR_CUDA;
     void *blob = nullptr;
     if (cudaMalloc(&blob, total) != cudaSuccess) return BCA_ERR_NO_MEMORY;
@@ -72,8 +76,14 @@ int upload(bca::Plan &P) {
     P.d_items = static_cast<const Item *>(put(P.items.data(), P.items.size() * sizeof(Item), s_items));
     P.d_pos = static_cast<const uint32_t *>(put(P.pos.data(), P.pos.size() * sizeof(uint32_t), s_pos));
     P.d_rope = static_cast<const float *>(put(P.rope.data(), P.rope.size() * sizeof(float), s_rope));
+    P.d_col_off = static_cast<const int32_t *>(put(P.col_off.data(), P.col_off.size() * sizeof(int32_t), s_coloff));
+    P.d_col_runs = static_cast<const Run *>(put(P.col_runs.data(), P.col_runs.size() * sizeof(Run), s_colruns));
+    P.d_bwd_items =
+        static_cast<const int32_t *>(put(P.bwd_items.data(), P.bwd_items.size() * sizeof(int32_t), s_bitems));
     P.d_status = static_cast<int *>(static_cast<void *>(b + off));
-    if (!P.d_run_off || !P.d_runs || !P.d_masks || !P.d_items || !P.d_pos || !P.d_rope) return BCA_ERR_CUDA;
+    if (!P.d_run_off || !P.d_runs || !P.d_masks || !P.d_items || !P.d_pos || !P.d_rope || !P.d_col_off ||
+        !P.d_col_runs || !P.d_bwd_items)
+        return BCA_ERR_CUDA;
     if (cudaMemset(P.d_status, 0, sizeof(int)) != cudaSuccess) return BCA_ERR_CUDA;
     return BCA_OK;
 }
@@ -156,6 +166,11 @@ int bca_plan_get_info(bca_plan_t plan, bca_plan_info *info) {
 int bca_plan_expand_rows(bca_plan_t plan, int64_t row_begin, int64_t row_end, uint8_t *out) {
     if (!plan) return BCA_ERR_INVALID_ARGUMENT;
     return bca::expand_rows(plan->plan, row_begin, row_end, out);
+}
+
+int bca_plan_expand_cols(bca_plan_t plan, int64_t key_begin, int64_t key_end, uint8_t *out) {
+    if (!plan) return BCA_ERR_INVALID_ARGUMENT;
+    return bca::expand_cols(plan->plan, key_begin, key_end, out);
 }
 
 size_t bca_workspace_bytes(bca_plan_t plan, int pass) {

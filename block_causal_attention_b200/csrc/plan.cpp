@@ -224,6 +224,52 @@ int compile_plan(Plan &P) {
     }
     P.run_off[P.nqt] = (int32_t)P.runs.size();
 
+    // ---- transposed runs for the backward (k-tile -> q-tiles), built by a
+    //      counting pass over the forward runs in q-tile order ----
+    {
+        std::vector<int64_t> cnt(P.nkt + 1, 0);
+        for (const Run &r : P.runs)
+            for (int32_t t = r.kt_begin; t < r.kt_end; ++t) cnt[t + 1]++;
+        for (int64_t t = 0; t < P.nkt; ++t) cnt[t + 1] += cnt[t];
+        std::vector<int64_t> fill(cnt.begin(), cnt.end() - 1);
+        std::vector<int32_t> ent_qt((size_t)cnt[P.nkt]), ent_mask((size_t)cnt[P.nkt]);
+        for (int64_t qt = 0; qt < P.nqt; ++qt)
+            for (int32_t ri = P.run_off[qt]; ri < P.run_off[qt + 1]; ++ri) {
+                const Run &r = P.runs[ri];
+                for (int32_t t = r.kt_begin; t < r.kt_end; ++t) {
+                    const int64_t at = fill[t]++;
+                    ent_qt[at] = (int32_t)qt;
+                    ent_mask[at] = r.mask_idx;
+                }
+            }
+        P.col_off.assign(P.nkt + 1, 0);
+        P.kt_qtiles.assign(P.nkt, 0);
+        P.col_runs.clear();
+        for (int64_t t = 0; t < P.nkt; ++t) {
+            P.col_off[t] = (int32_t)P.col_runs.size();
+            for (int64_t e = cnt[t]; e < cnt[t + 1]; ++e) {
+                const int32_t qt = ent_qt[e], mk = ent_mask[e];
+                if (mk < 0 && !P.col_runs.empty() && (int64_t)P.col_off[t] < (int64_t)P.col_runs.size() &&
+                    P.col_runs.back().mask_idx < 0 && P.col_runs.back().kt_end == qt)
+                    P.col_runs.back().kt_end = qt + 1;
+                else
+                    P.col_runs.push_back({qt, qt + 1, mk, 0});
+            }
+            P.kt_qtiles[t] = (int32_t)(cnt[t + 1] - cnt[t]);
+        }
+        P.col_off[P.nkt] = (int32_t)P.col_runs.size();
+        P.bwd_items.resize((size_t)P.nkt * P.hkv);
+        for (int64_t t = 0; t < P.nkt; ++t)
+            for (int g = 0; g < P.hkv; ++g) P.bwd_items[t * P.hkv + g] = (int32_t)(t * P.hkv + g);
+        std::stable_sort(P.bwd_items.begin(), P.bwd_items.end(), [&](int32_t x, int32_t y) {
+            const int32_t cx = P.kt_qtiles[x / P.hkv], cy = P.kt_qtiles[y / P.hkv];
+            if (cx != cy) return cx > cy;
+            const int gx = x % P.hkv, gy = y % P.hkv;
+            if (gx != gy) return gx < gy;
+            return x < y;
+        });
+    }
+
     // ---- items, longest first; ties grouped by KV group then q-tile so that CTAs
     //      running together stream the same K/V tiles ----
     const int npairs = P.hq / 2, G = P.hq / P.hkv;
@@ -296,6 +342,29 @@ int expand_rows(const Plan &P, int64_t r0, int64_t r1, uint8_t *out) {
                         if (key >= P.nk) return BCA_ERR_BAD_SLICE;  // a compiled key out of range
                         row[key] = (uint8_t)(row[key] + 1);
                     }
+                }
+            }
+        }
+    }
+    return BCA_OK;
+}
+
+int expand_cols(const Plan &P, int64_t k0, int64_t k1, uint8_t *out) {
+    if (k0 < 0 || k1 < k0 || k1 > P.nk || !out) return BCA_ERR_INVALID_ARGUMENT;
+    std::memset(out, 0, (size_t)(k1 - k0) * (size_t)P.nq);
+    for (int64_t j = k0; j < k1; ++j) {
+        const int64_t kt = j / kTileK;
+        const int c = (int)(j - kt * kTileK);
+        uint8_t *col = out + (size_t)(j - k0) * (size_t)P.nq;
+        for (int32_t ri = P.col_off[kt]; ri < P.col_off[kt + 1]; ++ri) {
+            const Run &run = P.col_runs[ri];
+            for (int32_t qt = run.kt_begin; qt < run.kt_end; ++qt) {
+                for (int r = 0; r < kTileQ; ++r) {
+                    const int64_t q = (int64_t)qt * kTileQ + r;
+                    if (q >= P.nq) break;
+                    const bool vis = run.mask_idx < 0 ||
+                                     ((P.masks[((size_t)run.mask_idx * kTileQ + r) * 4 + c / 32] >> (c % 32)) & 1u);
+                    if (vis) col[q] = (uint8_t)(col[q] + 1);
                 }
             }
         }

@@ -43,6 +43,13 @@ struct Plan {
     std::vector<int32_t> qt_tiles;   // k-tiles per q-tile
     int64_t visible_pairs = 0, nfull = 0, npartial = 0;
 
+    // transposed view for the backward: per k-tile, runs of q-tiles that see it
+    // (Run.kt_begin/kt_end hold the q-tile range here; a partial tile is its own run)
+    std::vector<int32_t> col_off;    // [nkt + 1]
+    std::vector<Run> col_runs;
+    std::vector<int32_t> kt_qtiles;  // q-tiles per k-tile
+    std::vector<int32_t> bwd_items;  // k-tile * hkv + kv head, longest-first
+
     // schedule and prologue tables
     std::vector<Item> items;         // longest-first
     std::vector<uint32_t> pos;       // packed (t << 16 | h << 8 | w) per new token
@@ -57,6 +64,9 @@ struct Plan {
     const Run *d_runs = nullptr;
     const uint32_t *d_masks = nullptr;
     const Item *d_items = nullptr;
+    const int32_t *d_col_off = nullptr;
+    const Run *d_col_runs = nullptr;
+    const int32_t *d_bwd_items = nullptr;
     const uint32_t *d_pos = nullptr;
     const float *d_rope = nullptr;
     int *d_status = nullptr;
@@ -76,5 +86,7 @@ int validate_problem(const bca_problem *p, Plan &plan);
 int compile_plan(Plan &plan);
 // Expand compiled tiles of rows [r0, r1) into a coverage map (host).
 int expand_rows(const Plan &plan, int64_t r0, int64_t r1, uint8_t *out);
+// Same from the transposed (backward) runs, for keys [k0, k1): out[(j - k0) * nq + i].
+int expand_cols(const Plan &plan, int64_t k0, int64_t k1, uint8_t *out);
 
 }  // namespace bca

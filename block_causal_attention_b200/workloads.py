@@ -194,6 +194,10 @@ WORKLOADS = {
                                 backward=True,
                                 description="40 chunks x 64 (1x8x8), KV range 16, "
                                             "transitions at 12/24/36"),
+    # one KV group of the 720p pipelined workload (16 query heads / 1 KV head): the
+    # same per-head work and mask at 1/8 of the size, for kernel profiling
+    "p720_1group": _c3_like("p720_1group", 3, 6, 45, 80, 16, 1,
+                            description="p720_pipelined restricted to one KV group"),
     "b45_replica": _wl("b45_replica", 12, 32, 2, 24, [Video(4, 2, 8, 12)],
                        description="4 chunks x 192 (2x8x12), D=24"),
 }

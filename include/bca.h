@@ -133,6 +133,11 @@ int bca_plan_get_info(bca_plan_t plan, bca_plan_info *info);
  * mark pair (i, j) visible (0 or 1 for a correct plan).  Host only. */
 int bca_plan_expand_rows(bca_plan_t plan, int64_t row_begin, int64_t row_end, uint8_t *out);
 
+/* The same from the backward's transposed tables (for each key tile, the runs of
+ * query tiles that see it), for keys [key_begin, key_end):
+ * out[(j - key_begin) * Nq + i].  Host only. */
+int bca_plan_expand_cols(bca_plan_t plan, int64_t key_begin, int64_t key_end, uint8_t *out);
+
 /* Bytes of caller-provided device workspace a pass needs (16-byte aligned). */
 size_t bca_workspace_bytes(bca_plan_t plan, int pass);
 

@@ -48,6 +48,29 @@ def test_compiled_mask_equals_oracle_mask(name):
     assert p.info()["visible_pairs"] == int(want.sum())
 
 
+@pytest.mark.parametrize("name", ["tiny", "b45_replica", "p720_replica", "packed_replica",
+                                  "kvrange_replica"])
+def test_transposed_tables_equal_oracle_mask(name):
+    """The backward's per-key-tile runs cover exactly the oracle's mask columns."""
+    w = W.WORKLOADS[name]
+    p = _plan(w)
+    got = p.expand_cols(0, w.nk)
+    want = oracle.mask_dense(w.slices_array(), w.nq, w.nk).T
+    assert got.max() <= 1
+    assert np.array_equal(got.astype(bool), want)
+
+
+@pytest.mark.parametrize("name", ["p720_pipelined", "packed_varlen", "long_kvrange"])
+def test_transposed_tables_full_size_columns(name):
+    w = W.WORKLOADS[name]
+    p = _plan(w)
+    rng = np.random.default_rng(3)
+    for j in list(rng.choice(w.nk, 6, replace=False)) + [0, w.nk - 1]:
+        got = p.expand_cols(int(j), int(j) + 1)[0]
+        assert got.max() <= 1
+        assert np.array_equal(got.astype(bool), oracle.mask_col(w.slices_array(), w.nq, int(j))), j
+
+
 @pytest.mark.parametrize("name", ["p720_pipelined", "packed_varlen", "long_kvrange"])
 def test_compiled_mask_full_size_rows(name):
     w = W.WORKLOADS[name]
@@ -79,6 +102,9 @@ def test_compiled_mask_random_slices():
         want = oracle.mask_dense(sl, nq, nk)
         assert got.max(initial=0) <= 1, trial
         assert np.array_equal(got.astype(bool), want), trial
+        gotc = p.expand_cols(0, nk)
+        assert gotc.max(initial=0) <= 1, trial
+        assert np.array_equal(gotc.astype(bool), want.T), trial
 
 
 def test_default_slices_are_block_causal():
