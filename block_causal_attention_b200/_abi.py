@@ -20,6 +20,8 @@ BCA_ERR_CUDA = -5
 BCA_ERR_DEVICE_TIMEOUT = -6
 BCA_ERR_HOST_ONLY_PLAN = -7
 BCA_ERR_NO_MEMORY = -8
+BCA_ERR_TOO_LARGE = -9
+BCA_STATIC_WORKSPACE_BYTES = 16 << 20
 
 BCA_SLICE_FULL = 0
 BCA_SLICE_CAUSAL = 1
@@ -31,8 +33,8 @@ BCA_PASS_BWD = 1
 # every symbol include/bca.h declares
 EXPORTS = ("bca_plan_create", "bca_plan_destroy", "bca_plan_get_info", "bca_plan_expand_rows",
            "bca_plan_expand_cols",
-           "bca_workspace_bytes", "bca_fwd", "bca_profile_enable", "bca_profile_read", "bca_status",
-           "bca_error_string")
+           "bca_workspace_bytes", "bca_fwd", "bca_fwd_static_workspace", "bca_profile_enable",
+           "bca_profile_read", "bca_status", "bca_error_string")
 BCA_KERNEL_KV_IMAGE = 0
 BCA_KERNEL_FWD = 1
 KERNEL_NAMES = {BCA_KERNEL_KV_IMAGE: "kv_image_kernel", BCA_KERNEL_FWD: "fwd_kernel"}
@@ -97,6 +99,8 @@ def lib() -> ctypes.CDLL:
         L.bca_workspace_bytes.restype = ctypes.c_size_t
         L.bca_fwd.argtypes = [vp] * 12
         L.bca_fwd.restype = i32
+        L.bca_fwd_static_workspace.argtypes = [vp] * 11
+        L.bca_fwd_static_workspace.restype = i32
         L.bca_profile_enable.argtypes = [vp, i32]
         L.bca_profile_enable.restype = i32
         L.bca_profile_read.argtypes = [vp, i32, ctypes.POINTER(i64), ctypes.POINTER(ctypes.c_double)]

@@ -9,10 +9,6 @@
 #include "kernels.hpp"
 #include "plan.hpp"
 
-struct bca_plan_s {
-    bca::Plan plan;
-};
-
 namespace bca {
 
 ProfScope::ProfScope(Plan &p, int k, cudaStream_t s) : plan(p), kernel(k), stream(s) {
@@ -255,6 +251,7 @@ const char *bca_error_string(int code) {
         case BCA_ERR_DEVICE_TIMEOUT: return "a device-side wait timed out";
         case BCA_ERR_HOST_ONLY_PLAN: return "plan was built host-only (BCA_PLAN_HOST_ONLY)";
         case BCA_ERR_NO_MEMORY: return "out of memory";
+        case BCA_ERR_TOO_LARGE: return "problem needs more scratch than the static workspace holds";
         default: return "unknown error";
     }
 }

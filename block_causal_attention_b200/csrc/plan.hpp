@@ -90,3 +90,8 @@ int expand_rows(const Plan &plan, int64_t r0, int64_t r1, uint8_t *out);
 int expand_cols(const Plan &plan, int64_t k0, int64_t k1, uint8_t *out);
 
 }  // namespace bca
+
+// The opaque handle behind bca_plan_t.
+struct bca_plan_s {
+    bca::Plan plan;
+};

@@ -63,6 +63,7 @@ extern "C" {
 #define BCA_ERR_DEVICE_TIMEOUT (-6)    /* a device-side wait ran out (see bca_status) */
 #define BCA_ERR_HOST_ONLY_PLAN (-7)    /* plan was built with BCA_PLAN_HOST_ONLY */
 #define BCA_ERR_NO_MEMORY (-8)         /* host or device allocation failed in bca_plan_create */
+#define BCA_ERR_TOO_LARGE (-9)         /* problem needs more scratch than the static workspace holds */
 
 /* AttnSlice type */
 #define BCA_SLICE_FULL 0
@@ -148,6 +149,32 @@ size_t bca_workspace_bytes(bca_plan_t plan, int pass);
 int bca_fwd(bca_plan_t plan, const void *q, const void *k, const void *v,
             const void *k_cache, const void *v_cache, const float *q_gain,
             const float *k_gain, void *o, float *lse, void *workspace, void *stream);
+
+/* Forward without a caller-provided workspace, for callers that may not allocate
+ * device memory themselves: for example a plug-in running inside a host process
+ * whose allocator owns all device memory and forbids raw allocations from library
+ * code, or a C caller with no allocator of its own on this path.  (The pages have
+ * no counterpart: this is a property of the library, not of the method.)
+ *
+ * Same arguments, layouts and results as bca_fwd, minus `workspace`.  The scratch
+ * that bca_fwd takes from the workspace (the K-hat and V tile images) lives instead
+ * in one file-scope device array of BCA_STATIC_WORKSPACE_BYTES that every GPU which
+ * loads the library holds until the process exits.  The call allocates nothing.
+ *  - Limit: problems whose bca_workspace_bytes(plan, BCA_PASS_FWD) exceeds
+ *    BCA_STATIC_WORKSPACE_BYTES are rejected with BCA_ERR_TOO_LARGE, before any
+ *    launch.  (16 MiB holds, e.g., 6144 keys x 8 KV heads at head_dim 48.)
+ *  - The first call on a device looks up the array's device address once (with
+ *    that device current); make that first call before any stream capture begins.
+ *  - Every call on a device shares the one array and leaves its contents behind.
+ *    Each call rewrites every byte it reads before reading it, so nothing needs to
+ *    start at zero, but calls whose kernels overlap on the GPU (other streams, or
+ *    other threads) race on it: serialise them.
+ *  - Per-kernel profiling (bca_profile_enable) creates CUDA events; the call
+ *    returns BCA_ERR_INVALID_ARGUMENT while it is enabled on the plan. */
+#define BCA_STATIC_WORKSPACE_BYTES (16u << 20)
+int bca_fwd_static_workspace(bca_plan_t plan, const void *q, const void *k, const void *v,
+                             const void *k_cache, const void *v_cache, const float *q_gain,
+                             const float *k_gain, void *o, float *lse, void *stream);
 
 /* Kernel kinds for per-kernel timing */
 #define BCA_KERNEL_KV_IMAGE 0  /* K-hat prologue + K/V tile images */

@@ -178,6 +178,6 @@ def test_empty_problem():
 
 
 def test_error_strings():
-    for c in range(0, -9, -1):
+    for c in range(0, -10, -1):
         assert _abi.error_string(c) != "unknown error"
     assert _abi.error_string(-100) == "unknown error"

@@ -1,0 +1,69 @@
+"""The allocation-free forward, bca_fwd_static_workspace, against bca_fwd.
+
+Some callers cannot allocate device memory on their own (a plug-in inside a host
+whose allocator owns all device memory, or a C caller without an allocator), so
+they cannot supply bca_fwd's workspace; bca_fwd_static_workspace keeps that scratch
+in a fixed device array inside the library instead.  These tests call it through
+the C ABI and check, on consecutive calls that share that array, that it gives the
+same results as bca_fwd within the tolerances of the other parity tests.  This
+file is collected last on purpose."""
+import numpy as np
+import pytest
+import torch
+
+from block_causal_attention_b200 import Plan, _abi
+from block_causal_attention_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+O_MAX, O_MEAN, LSE_MAX = 1e-2, 1e-3, 1e-3
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _static_fwd(plan, x, o, lse):
+    rc = _abi.lib().bca_fwd_static_workspace(plan._h, _ptr(x["q"]), _ptr(x["k"]), _ptr(x["v"]),
+                                             _ptr(x["k_cache"]), _ptr(x["v_cache"]), None, None,
+                                             _ptr(o), _ptr(lse), torch.cuda.current_stream().cuda_stream)
+    assert rc == _abi.BCA_OK, _abi.error_string(rc)
+    torch.cuda.synchronize()
+    assert plan.status() == _abi.BCA_OK
+
+
+def _close(o, lse, o_ref, lse_ref):
+    fin = torch.isfinite(lse_ref)
+    assert torch.equal(torch.isfinite(lse), fin)
+    eo = (o.double() - o_ref.double()).abs()
+    el = (lse[fin].double() - lse_ref[fin].double()).abs()
+    assert eo.max().item() <= O_MAX and eo.mean().item() <= O_MEAN
+    assert el.max().item() <= LSE_MAX
+
+
+def test_static_workspace_matches_bca_fwd_on_consecutive_calls():
+    runs = []
+    for name in ("p720_replica", "b45_replica"):
+        w = W.WORKLOADS[name]
+        x = W.make_inputs(w, "cuda")
+        plan = Plan.from_workload(w)
+        assert plan.workspace_bytes() <= _abi.BCA_STATIC_WORKSPACE_BYTES
+        o_ref, lse_ref = plan.fwd(x["q"], x["k"], x["v"], x["k_cache"], x["v_cache"])
+        torch.cuda.synchronize()
+        runs.append((plan, x, o_ref, lse_ref))
+    # two calls in a row on the same problem, then one on a different problem (other
+    # head_dim and key count) that reuses the same static array, then the first again
+    for plan, x, o_ref, lse_ref in (runs[0], runs[0], runs[1], runs[0]):
+        o = torch.full_like(o_ref, float("nan"))
+        lse = torch.full_like(lse_ref, float("nan"))
+        _static_fwd(plan, x, o, lse)
+        _close(o, lse, o_ref, lse_ref)
+
+
+def test_static_workspace_rejects_problems_beyond_its_size():
+    w = W.WORKLOADS["p720_pipelined"]
+    plan = Plan.from_workload(w)
+    assert plan.workspace_bytes() > _abi.BCA_STATIC_WORKSPACE_BYTES
+    rc = _abi.lib().bca_fwd_static_workspace(plan._h, *([None] * 10))
+    assert rc == _abi.BCA_ERR_TOO_LARGE
+    assert "static workspace" in _abi.error_string(rc)
