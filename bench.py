@@ -44,6 +44,7 @@ def _args():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "fwdbwd"], default="fwdbwd")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=8, help="query rows (all heads) in the oracle sample")
@@ -224,9 +225,22 @@ def run_ours(a):
     lse = torch.empty((hq, w.nq), device="cuda", dtype=torch.float32)
     ws = plan.alloc_workspace()
     stream = torch.cuda.current_stream()
+    bwd = a.pass_ == "fwdbwd"
+    if bwd:
+        do = shard(W.make_input(w, W.T_DO, "cuda"), h0, h1)
+        f32 = torch.float32
+        dq = torch.empty((w.nq, hq, w.d), device="cuda", dtype=f32)
+        dk = torch.empty((w.nq, hkv, w.d), device="cuda", dtype=f32)
+        dv = torch.empty((w.nq, hkv, w.d), device="cuda", dtype=f32)
+        dkc = torch.empty((w.num_cache_keys, hkv, w.d), device="cuda", dtype=f32) if w.num_cache_keys else None
+        dvc = torch.empty((w.num_cache_keys, hkv, w.d), device="cuda", dtype=f32) if w.num_cache_keys else None
+        wsb = plan.alloc_workspace(1)
 
     def step():
         plan.fwd(q, k, v, kc, vc, o=o, lse=lse, workspace=ws, stream=stream)
+        if bwd:
+            plan.bwd(q, k, v, kc, vc, o, lse, do, dq=dq, dk=dk, dv=dv, dk_cache=dkc, dv_cache=dvc, workspace=wsb,
+                     stream=stream)
 
     def barrier():
         torch.cuda.synchronize()
@@ -264,7 +278,8 @@ def run_ours(a):
         elapsed_ms = float(t.item())
 
     pairs = info["visible_pairs"]
-    flops_step_total = 4.0 * w.d * w.hq * pairs           # all ranks together
+    fwd_total = 4.0 * w.d * w.hq * pairs                  # all ranks together
+    flops_step_total = fwd_total * (3.5 if bwd else 1.0)  # bwd = 2.5 x fwd (five GEMMs vs two)
     flops_fwd_launch = 4.0 * w.d * hq * pairs            # this rank's launch
     value = flops_step_total * a.steps / (elapsed_ms * 1e-3) / 1e12
     tokens_per_s = w.nq * a.steps / (elapsed_ms * 1e-3)
@@ -277,22 +292,36 @@ def run_ours(a):
         hvc = vc.cpu().pin_memory() if vc is not None else None
         ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        dkc = torch.empty_like(kc) if kc is not None else None
-        dvc = torch.empty_like(vc) if vc is not None else None
+        if bwd:
+            hdo = do.cpu().pin_memory()
+            ddo = torch.empty_like(do)
+            hgrads = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv, dkc, dvc)
+                      if t is not None]
+        dq_, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dkc_ = torch.empty_like(kc) if kc is not None else None
+        dvc_ = torch.empty_like(vc) if vc is not None else None
         h2d = sum(t.numel() * t.element_size() for t in (hq_, hk_, hv_, hkc, hvc) if t is not None)
         d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+        if bwd:
+            h2d += hdo.numel() * hdo.element_size()
+            d2h += sum(t.numel() * t.element_size() for t in hgrads)
 
         def e2e_step():
-            dq.copy_(hq_, non_blocking=True)
-            dk.copy_(hk_, non_blocking=True)
-            dv.copy_(hv_, non_blocking=True)
-            if dkc is not None:
-                dkc.copy_(hkc, non_blocking=True)
-                dvc.copy_(hvc, non_blocking=True)
-            plan.fwd(dq, dk, dv, dkc, dvc, o=o, lse=lse, workspace=ws, stream=stream)
+            dq_.copy_(hq_, non_blocking=True)
+            dk_.copy_(hk_, non_blocking=True)
+            dv_.copy_(hv_, non_blocking=True)
+            if dkc_ is not None:
+                dkc_.copy_(hkc, non_blocking=True)
+                dvc_.copy_(hvc, non_blocking=True)
+            plan.fwd(dq_, dk_, dv_, dkc_, dvc_, o=o, lse=lse, workspace=ws, stream=stream)
             ho.copy_(o, non_blocking=True)
             hl.copy_(lse, non_blocking=True)
+            if bwd:
+                ddo.copy_(hdo, non_blocking=True)
+                plan.bwd(dq_, dk_, dv_, dkc_, dvc_, o, lse, ddo, dq=dq, dk=dk, dv=dv, dk_cache=dkc, dv_cache=dvc,
+                         workspace=wsb, stream=stream)
+                for hdst, src in zip(hgrads, [t for t in (dq, dk, dv, dkc, dvc) if t is not None]):
+                    hdst.copy_(src, non_blocking=True)
 
         e2e_step()
         barrier()
@@ -314,21 +343,30 @@ def run_ours(a):
     # ---- roofline of the dominant kernel (the attention forward)
     peaks, peak_src = _peaks()
     n_fwd, ms_fwd = prof["fwd_kernel"]
-    n_img, ms_img = prof["kv_image_kernel"]
     avg_fwd_ms = ms_fwd / max(1, n_fwd)
-    achieved = flops_fwd_launch / (avg_fwd_ms * 1e-3) / 1e12
+    n_bwd, ms_bwd = prof["bwd_kernel"]
+    avg_bwd_ms = ms_bwd / max(1, n_bwd)
+    ms_all = sum(t for _, t in prof.values())
+    launches = sum(c for c, _ in prof.values())
+    if bwd and ms_bwd >= ms_fwd:
+        dom, dom_flops, dom_ms = "bwd_kernel", 2.5 * flops_fwd_launch, avg_bwd_ms
+    else:
+        dom, dom_flops, dom_ms = "fwd_kernel", flops_fwd_launch, avg_fwd_ms
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
         with open(tpath) as f:
-            traffic = json.load(f).get(f"fwd_kernel:{w.name}")
+            traffic = json.load(f).get(f"{dom}:{w.name}")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
                 "frac": achieved / peak_sus, "traffic": traffic,
-                "kernel": "fwd_kernel", "peak_kind": f"bf16 dense, sustained, {peak_src}",
+                "kernel": dom, "peak_kind": f"bf16 dense, sustained, {peak_src}",
                 "frac_of_burst_peak": achieved / peak_burst,
-                "kernel_share_of_step": ms_fwd / max(1e-9, ms_fwd + ms_img)}
+                "kernel_share_of_step": (ms_bwd if dom == "bwd_kernel" else ms_fwd) / max(1e-9, ms_all)}
+    fwd_tflops = flops_fwd_launch / (avg_fwd_ms * 1e-3) / 1e12
+    bwd_tflops = 2.5 * flops_fwd_launch / (avg_bwd_ms * 1e-3) / 1e12 if n_bwd else None
 
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
@@ -342,16 +380,19 @@ def run_ours(a):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": elapsed_ms / a.steps, "higher_is_better": True,
             "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "pass": "fwd", "nq": w.nq, "nk": w.nk, "hq": w.hq, "hkv": w.hkv,
+            "config": {"workload": w.name, "pass": a.pass_, "nq": w.nq, "nk": w.nk, "hq": w.hq, "hkv": w.hkv,
                        "d": w.d, "visible_pairs_per_head": pairs,
                        "parallelism": f"head-parallel x{world}" if world > 1 else "1 GPU",
                        "l2": "inputs larger than L2 (Q 1.06 GB, K/V images 0.4 GB, O 1.06 GB)",
                        "plan_compile_ms": plan_ms, "tokens_per_s": tokens_per_s,
                        "pct_peak_sustained": 100 * value / peak_sus / world,
-                       "pct_peak_burst": 100 * value / peak_burst / world},
+                       "pct_peak_burst": 100 * value / peak_burst / world,
+                       "fwd_kernel_tflops": fwd_tflops, "bwd_kernel_tflops": bwd_tflops,
+                       "fwd_kernel_pct_sustained": 100 * fwd_tflops / peak_sus,
+                       "bwd_kernel_pct_sustained": (100 * bwd_tflops / peak_sus) if bwd_tflops else None},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-            "gpu_launches": int(n_fwd + n_img),
-            "kernel_ms": {"fwd_kernel": avg_fwd_ms, "kv_image_kernel": ms_img / max(1, n_img)},
+            "gpu_launches": int(launches),
+            "kernel_ms": {k: (t / c if c else None) for k, (c, t) in prof.items()},
         }
         print(json.dumps(line), flush=True)
     plan.close()

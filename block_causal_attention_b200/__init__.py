@@ -115,6 +115,33 @@ class Plan:
         _abi.check(rc, "bca_fwd")
         return o, lse
 
+    def bwd(self, q, k, v, k_cache, v_cache, o, lse, dout, *, dq=None, dk=None, dv=None, dk_cache=None,
+            dv_cache=None, workspace=None, q_gain=None, k_gain=None, stream=None, want_cache_grads=True):
+        """Gradients (fp32) w.r.t. q, k, v (new tokens, through QK-Norm + RoPE) and the
+        cache; o, lse are the forward's outputs, dout the upstream gradient of O."""
+        import torch
+        if self.host_only:
+            raise BcaError(_abi.BCA_ERR_HOST_ONLY_PLAN, "bwd")
+        if dout.dtype != torch.bfloat16 or tuple(dout.shape) != (self.nq, self.hq, self.d) or \
+                not dout.is_contiguous():
+            raise ValueError("dout: expected contiguous bf16 [Nq, Hq, D]")
+        dev = q.device
+        f32 = torch.float32
+        dq = torch.empty((self.nq, self.hq, self.d), device=dev, dtype=f32) if dq is None else dq
+        dk = torch.empty((self.nq, self.hkv, self.d), device=dev, dtype=f32) if dk is None else dk
+        dv = torch.empty((self.nq, self.hkv, self.d), device=dev, dtype=f32) if dv is None else dv
+        if self.num_cache_keys and want_cache_grads:
+            shp = (self.num_cache_keys, self.hkv, self.d)
+            dk_cache = torch.empty(shp, device=dev, dtype=f32) if dk_cache is None else dk_cache
+            dv_cache = torch.empty(shp, device=dev, dtype=f32) if dv_cache is None else dv_cache
+        if workspace is None:
+            workspace = self.alloc_workspace(_abi.BCA_PASS_BWD)
+        rc = self._lib.bca_bwd(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(q_gain),
+                               _ptr(k_gain), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                               _ptr(dk_cache), _ptr(dv_cache), _ptr(workspace), self._stream(stream))
+        _abi.check(rc, "bca_bwd")
+        return dq, dk, dv, dk_cache, dv_cache
+
     def profile(self, enable: bool = True) -> None:
         """Bracket every kernel launched for this plan with CUDA events."""
         _abi.check(self._lib.bca_profile_enable(self._h, 1 if enable else 0), "bca_profile_enable")

@@ -33,11 +33,12 @@ BCA_PASS_BWD = 1
 # every symbol include/bca.h declares
 EXPORTS = ("bca_plan_create", "bca_plan_destroy", "bca_plan_get_info", "bca_plan_expand_rows",
            "bca_plan_expand_cols",
-           "bca_workspace_bytes", "bca_fwd", "bca_fwd_static_workspace", "bca_profile_enable",
+           "bca_workspace_bytes", "bca_fwd", "bca_fwd_static_workspace", "bca_bwd", "bca_profile_enable",
            "bca_profile_read", "bca_status", "bca_error_string")
 BCA_KERNEL_KV_IMAGE = 0
 BCA_KERNEL_FWD = 1
-KERNEL_NAMES = {BCA_KERNEL_KV_IMAGE: "kv_image_kernel", BCA_KERNEL_FWD: "fwd_kernel"}
+KERNEL_NAMES = {0: "kv_image_kernel", 1: "fwd_kernel", 2: "bwd_prep_kernel", 3: "bwd_kv_image_kernel",
+                4: "bwd_kernel", 5: "bwd_dq_kernel"}
 
 
 class bca_slice(ctypes.Structure):
@@ -99,6 +100,8 @@ def lib() -> ctypes.CDLL:
         L.bca_workspace_bytes.restype = ctypes.c_size_t
         L.bca_fwd.argtypes = [vp] * 12
         L.bca_fwd.restype = i32
+        L.bca_bwd.argtypes = [vp] * 18
+        L.bca_bwd.restype = i32
         L.bca_fwd_static_workspace.argtypes = [vp] * 11
         L.bca_fwd_static_workspace.restype = i32
         L.bca_profile_enable.argtypes = [vp, i32]

@@ -172,6 +172,7 @@ int bca_plan_expand_cols(bca_plan_t plan, int64_t key_begin, int64_t key_end, ui
 size_t bca_workspace_bytes(bca_plan_t plan, int pass) {
     if (!plan) return 0;
     if (pass == BCA_PASS_FWD) return bca::fwd_workspace_bytes(plan->plan);
+    if (pass == BCA_PASS_BWD) return bca::bwd_workspace_bytes(plan->plan);
     return 0;
 }
 
@@ -190,6 +191,32 @@ int bca_fwd(bca_plan_t plan, const void *q, const void *k, const void *v, const 
         if (p && !aligned16(p)) return BCA_ERR_MISALIGNED;
     bca::FwdIO io{q, k, v, k_cache, v_cache, q_gain, k_gain, o, lse, workspace};
     return bca::launch_fwd(P, io, static_cast<cudaStream_t>(stream));
+}
+
+int bca_bwd(bca_plan_t plan, const void *q, const void *k, const void *v, const void *k_cache,
+            const void *v_cache, const float *q_gain, const float *k_gain, const void *o, const float *lse,
+            const void *dout, float *dq, float *dk, float *dv, float *dk_cache, float *dv_cache,
+            void *workspace, void *stream) {
+    if (!plan) return BCA_ERR_INVALID_ARGUMENT;
+    bca::Plan &P = plan->plan;
+    int rc = check_device(P);
+    if (rc != BCA_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (P.nq == 0) {
+        // no query: every gradient is zero
+        const size_t cb = (size_t)P.nc * P.hkv * P.d * sizeof(float);
+        if (dk_cache && cudaMemsetAsync(dk_cache, 0, cb, s) != cudaSuccess) return BCA_ERR_CUDA;
+        if (dv_cache && cudaMemsetAsync(dv_cache, 0, cb, s) != cudaSuccess) return BCA_ERR_CUDA;
+        return BCA_OK;
+    }
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return BCA_ERR_INVALID_ARGUMENT;
+    if (P.nc > 0 && (!k_cache || !v_cache)) return BCA_ERR_INVALID_ARGUMENT;
+    const void *ptrs[] = {q, k, v, k_cache, v_cache, q_gain, k_gain, o, lse, dout, dq, dk, dv, dk_cache, dv_cache,
+                          workspace};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return BCA_ERR_MISALIGNED;
+    bca::BwdIO io{q, k, v, k_cache, v_cache, q_gain, k_gain, o, lse, dout, dq, dk, dv, dk_cache, dv_cache, workspace};
+    return bca::launch_bwd(P, io, s);
 }
 
 int bca_profile_enable(bca_plan_t plan, int enable) {

@@ -1,0 +1,798 @@
+// Backward pass of block-causal GQA attention on sm_100a.
+//
+//   bwd_prep_kernel    : per (query tile, query head): Q-hat (QK-Norm + RoPE, scaled by
+//                        log2(e)/sqrt(D)) as an fp16 image, bit-identical to the forward's
+//                        Q tile, so S and hence P are recomputed exactly as the forward saw
+//                        them; dO as a bf16 image; LSE in log2 units; Dsum_i = dO_i . O_i;
+//                        the largest |dO_i|; zeroes the dQ rows.
+//   bwd_kv_image_kernel: K-hat (fp16, as in the forward) and V (bf16) images in the
+//                        key-row core layout, and the largest |v_j|.
+//   Precision: dP^T = V dO^T and dV = P^T dO run on bf16 (exact inputs; P rounded to
+//   bf16).  dS feeds dK = dS^T Q and dQ = dS K as fp16 against the fp16 Q-hat / K-hat
+//   (11-bit significands, 4x finer than bf16).  fp16's range is made safe by a
+//   power-of-two scale on dS chosen from |dS| <= 2 max|dO_i| max|v_j| (Cauchy-Schwarz;
+//   P <= 1 and |Dsum_i| <= |dO_i| max|v_j|), undone exactly on dK and dQ.
+//   bwd_kernel         : one CTA per (key tile, KV head).  It loops over every
+//                        (query tile, query head of the group) that sees the key tile, in
+//                        a fixed order, so dK and dV are accumulated deterministically
+//                        in tensor memory.  Per step it recomputes S^T = K Q^T and
+//                        dP^T = V dO^T, forms P^T = exp2(S^T - LSE) and
+//                        dS^T = P^T (dP^T - Dsum) in the compute warps, then issues
+//                        dV += P^T dO, dK += dS^T Q and dQ_part = dS K; dQ_part is added
+//                        to dQ with float4 atomics (the one non-deterministic sum).
+//   bwd_dq_kernel      : dQ <- prologue backward (RoPE^T, RMS-norm^T) of dQ-hat, in place.
+//
+// Gradients of the forward defined in fwd.cu; the pages give the forward only
+// (MAGI-1 research notes (zhao9797.github.io), "Infra > MagiAttention >
+// Flex-Flash-Attention" is used in training, hence the backward).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.hpp"
+#include "prologue.cuh"
+#include "sm100.cuh"
+
+namespace bca {
+
+using namespace sm100;
+
+namespace {
+
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.69314718055994531f;
+
+struct PrepArgs {
+    const __nv_bfloat16 *q, *dout;
+    const void *o;
+    int o_fp32;
+    const float *lse, *q_gain;
+    const uint32_t *pos;
+    const float *rope;
+    int32_t off0, off1, off2;
+    int64_t nq, nqt;
+    int hq;
+    float eps, qscale;
+    __half *qimg16;
+    __nv_bfloat16 *doimg;
+    float *lse2, *dsum, *dq;
+    float *bounds;  // [0] = max |dO_i| (atomic max on the float bits)
+};
+
+struct BwdKVArgs {
+    const __nv_bfloat16 *k, *v, *kc, *vc;
+    const float *k_gain;
+    const uint32_t *pos;
+    const float *rope;
+    int32_t off0, off1, off2;
+    int64_t nc, nk, nkt;
+    int hkv;
+    float eps;
+    __half *kimg16;
+    __nv_bfloat16 *vimg;
+    float *bounds;  // [1] = max |v_j|
+};
+
+struct BwdArgs {
+    const __half *kimg16, *qimg16;
+    const __nv_bfloat16 *vimg, *doimg;
+    const float *bounds;
+    const float *lse2, *dsum;
+    const int32_t *col_off;
+    const Run *col_runs;
+    const uint32_t *masks;
+    const int32_t *items;
+    const __nv_bfloat16 *k;
+    const float *k_gain;
+    const uint32_t *pos;
+    const float *rope;
+    int32_t off0, off1, off2;
+    int64_t nq, nk, nc, nqt, nkt;
+    int hq, hkv;
+    float eps;
+    float *dq, *dk, *dv, *dkc, *dvc;
+    int *status;
+};
+
+struct DqArgs {
+    const __nv_bfloat16 *q;
+    const float *q_gain;
+    const uint32_t *pos;
+    const float *rope;
+    int32_t off0, off1, off2;
+    int64_t nq;
+    int hq;
+    float eps, scale;
+    const float *bounds;
+    float *dq;
+};
+
+// Power-of-two scale applied to dS before its fp16 rounding: 1 unless the bound
+// 2 max|dO| max|v| on |dS| exceeds 2^14, else the power of two bringing it below.
+__device__ __forceinline__ float ds_scale(const float *bounds) {
+    const float b = 2.0f * __ldg(bounds) * __ldg(bounds + 1);
+    if (!(b > 16384.0f)) return 1.0f;
+    const float e = ceilf(log2f(b * (1.0f / 16384.0f)) + 1e-3f);
+    return exp2f(-fminf(e, 100.0f));
+}
+
+// atomic max of non-negative floats through their (order-preserving) bit patterns
+__device__ __forceinline__ void atomic_max_nonneg(float *addr, float v) {
+    atomicMax(reinterpret_cast<int *>(addr), __float_as_int(v));
+}
+
+// core-matrix image offset (in 16-byte chunks) of chunk c (8 columns) of row r in a
+// 128-row tile laid out [column group][row group][8 rows][8 columns]
+__device__ __forceinline__ int img_chunk(int c, int r) { return (c * 16 + r / 8) * 8 + (r % 8); }
+
+template <int D>
+__device__ __forceinline__ void load_row_f32(const float *src, float (&x)[D]) {
+    const float4 *s = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c) {
+        const float4 f = s[c];
+        x[4 * c] = f.x;
+        x[4 * c + 1] = f.y;
+        x[4 * c + 2] = f.z;
+        x[4 * c + 3] = f.w;
+    }
+}
+
+// ------------------------------------------------------------------ preparation
+
+template <int D>
+__global__ void __launch_bounds__(128) bwd_prep_kernel(PrepArgs a) {
+    constexpr int DPAD = Geo<D>::DPAD;
+    const int t = threadIdx.x;
+    const int64_t qt = blockIdx.x;
+    const int h = blockIdx.y;
+    const int64_t q = qt * 128 + t;
+    const bool live = q < a.nq;
+    const size_t tile = ((size_t)h * a.nqt + qt) * (128 * DPAD);
+    const size_t row = ((size_t)q * a.hq + h) * D;
+
+    float x[D];
+    if (live) {
+        load_row_bf16<D>(a.q + row, x);
+        qk_prologue<D>(x, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps, a.qscale);
+    } else {
+#pragma unroll
+        for (int d = 0; d < D; ++d) x[d] = 0.f;
+    }
+    uint4 *q16 = reinterpret_cast<uint4 *>(a.qimg16 + tile);
+#pragma unroll
+    for (int c = 0; c < DPAD / 8; ++c) q16[img_chunk(c, t)] = pack_chunk_f16<D>(x, c);
+
+    float g[D];
+    if (live) {
+        load_row_bf16<D>(a.dout + row, g);
+    } else {
+#pragma unroll
+        for (int d = 0; d < D; ++d) g[d] = 0.f;
+    }
+    uint4 *dob = reinterpret_cast<uint4 *>(a.doimg + tile);
+#pragma unroll
+    for (int c = 0; c < DPAD / 8; ++c) dob[img_chunk(c, t)] = pack_chunk_bf16<D>(g, c);
+    {
+        float n2 = 0.f;
+#pragma unroll
+        for (int d = 0; d < D; ++d) n2 = fmaf(g[d], g[d], n2);
+        float m = sqrtf(n2);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if ((t & 31) == 0) atomic_max_nonneg(a.bounds, m);
+    }
+
+    float dsum = 0.f, lse2 = INFINITY;
+    if (live) {
+        if (a.o_fp32) load_row_f32<D>(static_cast<const float *>(a.o) + row, x);
+        else load_row_bf16<D>(static_cast<const __nv_bfloat16 *>(a.o) + row, x);
+#pragma unroll
+        for (int d = 0; d < D; ++d) dsum = fmaf(g[d], x[d], dsum);
+        const float L = a.lse[(size_t)h * a.nq + q];
+        if (L > -INFINITY) lse2 = L * kLog2e;  // a row with no visible key keeps +inf: P = 0
+        float4 *dqr = reinterpret_cast<float4 *>(a.dq + row);
+#pragma unroll
+        for (int c = 0; c < D / 4; ++c) dqr[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    a.lse2[((size_t)h * a.nqt + qt) * 128 + t] = lse2;
+    a.dsum[((size_t)h * a.nqt + qt) * 128 + t] = dsum;
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) bwd_kv_image_kernel(BwdKVArgs a) {
+    constexpr int DPAD = Geo<D>::DPAD;
+    const int t = threadIdx.x;
+    const int64_t kt = blockIdx.x;
+    const int g = blockIdx.y;
+    const int64_t key = kt * 128 + t;
+    const size_t tile = ((size_t)g * a.nkt + kt) * (128 * DPAD);
+    float x[D];
+    if (key < a.nc) {
+        load_row_bf16<D>(a.kc + ((size_t)key * a.hkv + g) * D, x);
+    } else if (key < a.nk) {
+        const int64_t n = key - a.nc;
+        load_row_bf16<D>(a.k + ((size_t)n * a.hkv + g) * D, x);
+        qk_prologue<D>(x, __ldg(a.pos + n), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps, 1.0f);
+    } else {
+#pragma unroll
+        for (int d = 0; d < D; ++d) x[d] = 0.f;
+    }
+    uint4 *k16 = reinterpret_cast<uint4 *>(a.kimg16 + tile);
+#pragma unroll
+    for (int c = 0; c < DPAD / 8; ++c) k16[img_chunk(c, t)] = pack_chunk_f16<D>(x, c);
+    if (key < a.nc) {
+        load_row_bf16<D>(a.vc + ((size_t)key * a.hkv + g) * D, x);
+    } else if (key < a.nk) {
+        load_row_bf16<D>(a.v + ((size_t)(key - a.nc) * a.hkv + g) * D, x);
+    } else {
+#pragma unroll
+        for (int d = 0; d < D; ++d) x[d] = 0.f;
+    }
+    uint4 *vo = reinterpret_cast<uint4 *>(a.vimg + tile);
+#pragma unroll
+    for (int c = 0; c < DPAD / 8; ++c) vo[img_chunk(c, t)] = pack_chunk_bf16<D>(x, c);
+    float n2 = 0.f;
+#pragma unroll
+    for (int d = 0; d < D; ++d) n2 = fmaf(x[d], x[d], n2);
+    float m = sqrtf(n2);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((t & 31) == 0) atomic_max_nonneg(a.bounds + 1, m);
+}
+
+// ------------------------------------------------------------------ main kernel
+
+template <int D>
+struct BwdSmem {
+    static constexpr int DPAD = Geo<D>::DPAD;
+    static constexpr int TILE = 128 * DPAD * 2;
+    static constexpr int STAGES = 2;
+    static constexpr int OFF_K16 = 0;
+    static constexpr int OFF_V = TILE;
+    static constexpr int OFF_STAGE = 2 * TILE;
+    static constexpr int ST_Q16 = 0, ST_DO = TILE, ST_LSE = 2 * TILE, ST_DSUM = 2 * TILE + 512,
+                         ST_MASK = 2 * TILE + 1024;
+    static constexpr int STAGE_BYTES = 2 * TILE + 1024 + 2048;
+    static constexpr int OFF_PT = OFF_STAGE + STAGES * STAGE_BYTES;  // P^T, bf16 128x128
+    static constexpr int OFF_DST = OFF_PT + 32768;                    // dS^T, fp16 128x128
+    static constexpr int OFF_BAR = OFF_DST + 32768;
+    static constexpr int B_KV = 0, B_ST_FULL = 1, B_ST_EMPTY = 3, B_S_FULL = 5, B_S_FREE = 6, B_DS_READY = 7,
+                         B_PDS_FREE = 8, B_DQ_FULL = 9, B_DQ_FREE = 10, B_MMA_DONE = 11, NBAR = 12;
+    static constexpr int OFF_TMEM_PTR = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_ABORT = OFF_TMEM_PTR + 4;
+    static constexpr int BYTES = OFF_ABORT + 12;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 256, COL_DV = 320, COL_DK = 384;
+};
+
+// Walks (query tile, query head) items of one key tile: runs of query tiles, and
+// for each query tile every head of the KV group.
+struct ItemCursor {
+    const Run *r, *end;
+    int32_t qt;
+    int hh, G;
+    __device__ __forceinline__ ItemCursor(const Run *b, const Run *e, int g)
+        : r(b), end(e), qt(b < e ? b->kt_begin : 0), hh(0), G(g) {}
+    __device__ __forceinline__ void next() {
+        if (++hh < G) return;
+        hh = 0;
+        if (++qt >= r->kt_end) {
+            ++r;
+            if (r < end) qt = r->kt_begin;
+        }
+    }
+};
+
+__device__ __forceinline__ bool wait_abort(uint32_t bar, uint32_t parity, int *status, volatile int *abort_flag) {
+    if (*abort_flag) return false;
+    if (mbar_wait(bar, parity, kWaitTimeoutNs)) return true;
+    atomicOr(status, kStatusTimeout);
+    *abort_flag = 1;
+    return false;
+}
+
+__device__ __forceinline__ bool warp_wait_abort(uint32_t bar, uint32_t parity, int *status,
+                                                volatile int *abort_flag) {
+    const bool ok = wait_abort(bar, parity, status, abort_flag);
+    return __all_sync(0xffffffffu, ok);
+}
+
+template <int D>
+__global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
+    using L = BwdSmem<D>;
+    constexpr int DPAD = L::DPAD;
+    constexpr int STAGES = L::STAGES;
+    constexpr uint32_t IDESC_S = idesc_f32acc(128, 128, kFmtF16);     // S^T: fp16 K-hat, Q-hat
+    constexpr uint32_t IDESC_DP = idesc_f32acc(128, 128, kFmtBF16);   // dP^T: bf16 V, dO
+    constexpr uint32_t IDESC_DV = idesc_f32acc_major(128, DPAD, kFmtBF16, 0, 1);  // dV: B MN-major
+    constexpr uint32_t IDESC_DK = idesc_f32acc_major(128, DPAD, kFmtF16, 0, 1);   // dK: B MN-major
+    constexpr uint32_t IDESC_DQ = idesc_f32acc_major(128, DPAD, kFmtF16, 1, 1);   // dQ: A and B MN-major
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t sbase = smem_u32(smem);
+    auto bar = [&](int i) -> uint32_t { return sbase + L::OFF_BAR + 8u * (uint32_t)i; };
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::OFF_ABORT);
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + L::OFF_TMEM_PTR);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int32_t it = a.items[blockIdx.x];
+    const int64_t kt = it / a.hkv;
+    const int g = it % a.hkv;
+    const int G = a.hq / a.hkv;
+    const Run *rb = a.col_runs + a.col_off[kt];
+    const Run *re = a.col_runs + a.col_off[kt + 1];
+    int n = 0;
+    for (const Run *r = rb; r < re; ++r) n += (r->kt_end - r->kt_begin) * G;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(bar(L::B_KV), 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(bar(L::B_ST_FULL + s), 1);
+            mbar_init(bar(L::B_ST_EMPTY + s), 1);
+        }
+        mbar_init(bar(L::B_S_FULL), 1);
+        mbar_init(bar(L::B_S_FREE), 256);
+        mbar_init(bar(L::B_DS_READY), 256);
+        mbar_init(bar(L::B_PDS_FREE), 1);
+        mbar_init(bar(L::B_DQ_FULL), 1);
+        mbar_init(bar(L::B_DQ_FREE), 256);
+        mbar_init(bar(L::B_MMA_DONE), 1);
+        mbar_fence_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 2) {
+        tmem_alloc(smem_u32(tmem_ptr), L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_ptr;
+
+    if (warp == 0) {
+        // ------------------------------------------------ producer
+        if (lane == 0) {
+            const size_t ktile = ((size_t)g * a.nkt + kt) * (128 * DPAD);
+            mbar_arrive_expect_tx(bar(L::B_KV), 2 * L::TILE);
+            bulk_g2s(sbase + L::OFF_K16, a.kimg16 + ktile, L::TILE, bar(L::B_KV));
+            bulk_g2s(sbase + L::OFF_V, a.vimg + ktile, L::TILE, bar(L::B_KV));
+            int issued = 0;
+            ItemCursor cur(rb, re, G);
+            for (int i = 0; i < n; ++i, cur.next()) {
+                const int s = i % STAGES;
+                if (i >= STAGES &&
+                    !wait_abort(bar(L::B_ST_EMPTY + s), ((i / STAGES) - 1) & 1, a.status, abort_flag))
+                    break;
+                const int h = g * G + cur.hh;
+                const size_t qtile = ((size_t)h * a.nqt + cur.qt) * (128 * DPAD);
+                const size_t vtile = ((size_t)h * a.nqt + cur.qt) * 128;
+                const int mk = cur.r->mask_idx;
+                const uint32_t st = sbase + L::OFF_STAGE + s * L::STAGE_BYTES;
+                mbar_arrive_expect_tx(bar(L::B_ST_FULL + s), 2 * L::TILE + 1024 + (mk >= 0 ? 2048 : 0));
+                bulk_g2s(st + L::ST_Q16, a.qimg16 + qtile, L::TILE, bar(L::B_ST_FULL + s));
+                bulk_g2s(st + L::ST_DO, a.doimg + qtile, L::TILE, bar(L::B_ST_FULL + s));
+                bulk_g2s(st + L::ST_LSE, a.lse2 + vtile, 512, bar(L::B_ST_FULL + s));
+                bulk_g2s(st + L::ST_DSUM, a.dsum + vtile, 512, bar(L::B_ST_FULL + s));
+                if (mk >= 0) bulk_g2s(st + L::ST_MASK, a.masks + (size_t)mk * 512, 2048, bar(L::B_ST_FULL + s));
+                ++issued;
+            }
+            mbar_wait(bar(L::B_KV), 0, kWaitTimeoutNs);
+            for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+                mbar_wait(bar(L::B_ST_FULL + i % STAGES), (i / STAGES) & 1, kWaitTimeoutNs);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t k16 = sbase + L::OFF_K16, vb = sbase + L::OFF_V;
+            const uint32_t pt = sbase + L::OFF_PT, dst = sbase + L::OFF_DST;
+            auto stage = [&](int i) -> uint32_t { return sbase + L::OFF_STAGE + (i % STAGES) * L::STAGE_BYTES; };
+            // S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 128 queries, K = DPAD; all K-major)
+            auto issue_s_dp = [&](int i) {
+                const uint32_t st = stage(i);
+#pragma unroll
+                for (int kk = 0; kk < DPAD / 16; ++kk)
+                    mma_f16(tbase + L::COL_S, smem_desc(k16 + kk * 4096, 2048, 128),
+                            smem_desc(st + L::ST_Q16 + kk * 4096, 2048, 128), IDESC_S, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < DPAD / 16; ++kk)
+                    mma_f16(tbase + L::COL_DP, smem_desc(vb + kk * 4096, 2048, 128),
+                            smem_desc(st + L::ST_DO + kk * 4096, 2048, 128), IDESC_DP, kk > 0);
+            };
+            bool ok = wait_abort(bar(L::B_KV), 0, a.status, abort_flag);
+            if (ok && n > 0) ok = wait_abort(bar(L::B_ST_FULL), 0, a.status, abort_flag);
+            tc_fence_after();
+            if (ok && n > 0) {
+                issue_s_dp(0);
+                mma_commit(bar(L::B_S_FULL));
+            }
+            for (int i = 0; i < n && ok; ++i) {
+                const uint32_t st = stage(i);
+                if (i + 1 < n) {
+                    ok = wait_abort(bar(L::B_ST_FULL + (i + 1) % STAGES), ((i + 1) / STAGES) & 1, a.status,
+                                    abort_flag) &&
+                         wait_abort(bar(L::B_S_FREE), i & 1, a.status, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_s_dp(i + 1);
+                    mma_commit(bar(L::B_S_FULL));
+                }
+                ok = wait_abort(bar(L::B_DS_READY), i & 1, a.status, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                // dV += P^T dO and dK += dS^T Q (M = 128 keys, N = DPAD, K = 128 queries):
+                // A K-major from P^T / dS^T, B MN-major from the dO / Q image
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+                    mma_f16(tbase + L::COL_DV, smem_desc(pt + kk * 4096, 2048, 128),
+                            smem_desc(st + L::ST_DO + kk * 256, 128, 2048), IDESC_DV, acc);
+                    mma_f16(tbase + L::COL_DK, smem_desc(dst + kk * 4096, 2048, 128),
+                            smem_desc(st + L::ST_Q16 + kk * 256, 128, 2048), IDESC_DK, acc);
+                }
+                if (i > 0) {
+                    ok = wait_abort(bar(L::B_DQ_FREE), (i - 1) & 1, a.status, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                // dQ_part = dS K (M = 128 queries, N = DPAD, K = 128 keys): A MN-major from
+                // the dS^T buffer, B MN-major from the K image
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16(tbase + L::COL_DQ, smem_desc(dst + kk * 256, 128, 2048),
+                            smem_desc(k16 + kk * 256, 128, 2048), IDESC_DQ, kk > 0);
+                mma_commit(bar(L::B_DQ_FULL));
+                mma_commit(bar(L::B_ST_EMPTY + i % STAGES));
+                mma_commit(bar(L::B_PDS_FREE));
+            }
+            mma_commit(bar(L::B_MMA_DONE));
+            mbar_wait(bar(L::B_MMA_DONE), 0, kWaitTimeoutNs);
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ------------------------------------------------ P, dS and the epilogues
+        const int wg = (warp - 4) / 4;
+        const int quarter = warp % 4;
+        const int r = quarter * 32 + lane;  // key row of S^T / dP^T; query row of dQ_part
+        const int c0 = 64 * wg;             // this warpgroup's query columns
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        uint4 *ptb = reinterpret_cast<uint4 *>(smem + L::OFF_PT);
+        uint4 *dsb = reinterpret_cast<uint4 *>(smem + L::OFF_DST);
+        bool ok = true;
+        int prev_qt = 0, prev_h = 0;
+        const float sc = ds_scale(a.bounds);
+
+        auto dq_epilogue = [&](int j, int qt_j, int h_j) -> bool {
+            if (!warp_wait_abort(bar(L::B_DQ_FULL), j & 1, a.status, abort_flag)) return false;
+            tc_fence_after();
+            constexpr int HALF = DPAD / 2;
+            float v[HALF];
+#pragma unroll
+            for (int c = 0; c < HALF / 8; ++c) {
+                uint32_t r8[8];
+                tmem_ld8(tbase + lane_off + L::COL_DQ + wg * HALF + 8 * c, r8);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[8 * c + e] = __uint_as_float(r8[e]);
+            }
+            tc_fence_before();
+            mbar_arrive(bar(L::B_DQ_FREE));
+            const int64_t qrow = (int64_t)qt_j * 128 + r;
+            if (qrow < a.nq) {
+                float *dst = a.dq + ((size_t)qrow * a.hq + h_j) * D + wg * HALF;
+#pragma unroll
+                for (int c = 0; c < HALF / 4; ++c)
+                    if (wg * HALF + 4 * c < D)
+                        atomicAdd(reinterpret_cast<float4 *>(dst + 4 * c),
+                                  make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]));
+            }
+            return true;
+        };
+
+        ItemCursor cur(rb, re, G);
+        for (int i = 0; i < n; ++i, cur.next()) {
+            const int s = i % STAGES;
+            const int h = g * G + cur.hh;
+            const uint8_t *st = smem + L::OFF_STAGE + s * L::STAGE_BYTES;
+            ok = warp_wait_abort(bar(L::B_ST_FULL + s), (i / STAGES) & 1, a.status, abort_flag) &&
+                 warp_wait_abort(bar(L::B_S_FULL), i & 1, a.status, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            float sv[64], dp[64];
+            {
+                uint32_t u[64];
+                tmem_ld32(tbase + lane_off + L::COL_S + c0, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+                tmem_ld32(tbase + lane_off + L::COL_S + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(u[c]);
+                tmem_ld32(tbase + lane_off + L::COL_DP + c0, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+                tmem_ld32(tbase + lane_off + L::COL_DP + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 64; ++c) dp[c] = __uint_as_float(u[c]);
+            }
+            tc_fence_before();
+            mbar_arrive(bar(L::B_S_FREE));
+
+            const float *lse2 = reinterpret_cast<const float *>(st + L::ST_LSE) + c0;
+            const float *dsum = reinterpret_cast<const float *>(st + L::ST_DSUM) + c0;
+            const bool partial = cur.r->mask_idx >= 0;
+            const uint32_t *mask = reinterpret_cast<const uint32_t *>(st + L::ST_MASK);
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                float p = ex2(sv[c] - lse2[c]);
+                if (partial && !((mask[(c0 + c) * 4 + r / 32] >> (r % 32)) & 1u)) p = 0.f;
+                sv[c] = p;
+                dp[c] = p * (dp[c] - dsum[c]) * sc;
+            }
+            if (i > 0) {
+                ok = warp_wait_abort(bar(L::B_PDS_FREE), (i - 1) & 1, a.status, abort_flag);
+                if (!ok) break;
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int idx = img_chunk(c0 / 8 + k, r);
+                ptb[idx] = make_uint4(pack_bf16x2(sv[8 * k], sv[8 * k + 1]), pack_bf16x2(sv[8 * k + 2], sv[8 * k + 3]),
+                                      pack_bf16x2(sv[8 * k + 4], sv[8 * k + 5]),
+                                      pack_bf16x2(sv[8 * k + 6], sv[8 * k + 7]));
+                dsb[idx] = make_uint4(pack_f16x2(dp[8 * k], dp[8 * k + 1]), pack_f16x2(dp[8 * k + 2], dp[8 * k + 3]),
+                                      pack_f16x2(dp[8 * k + 4], dp[8 * k + 5]), pack_f16x2(dp[8 * k + 6], dp[8 * k + 7]));
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bar(L::B_DS_READY));
+            if (i > 0 && !dq_epilogue(i - 1, prev_qt, prev_h)) {
+                ok = false;
+                break;
+            }
+            prev_qt = cur.qt;
+            prev_h = h;
+        }
+        if (ok && n > 0) ok = dq_epilogue(n - 1, prev_qt, prev_h);
+
+        // dK / dV epilogue: warpgroup 0 writes dV, warpgroup 1 dK (through the
+        // prologue backward for new keys)
+        if (ok && n > 0) ok = warp_wait_abort(bar(L::B_MMA_DONE), 0, a.status, abort_flag);
+        tc_fence_after();
+        float acc[DPAD];
+#pragma unroll
+        for (int d = 0; d < DPAD; ++d) acc[d] = 0.f;
+        if (ok && n > 0) {
+#pragma unroll
+            for (int c = 0; c < DPAD / 8; ++c) {
+                uint32_t r8[8];
+                tmem_ld8(tbase + lane_off + (wg == 0 ? L::COL_DV : L::COL_DK) + 8 * c, r8);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[8 * c + e] = __uint_as_float(r8[e]);
+            }
+        }
+        const int64_t key = kt * 128 + r;
+        if (key < a.nk) {
+            if (wg == 0) {
+                float *dst = key < a.nc ? (a.dvc ? a.dvc + ((size_t)key * a.hkv + g) * D : nullptr)
+                                        : a.dv + ((size_t)(key - a.nc) * a.hkv + g) * D;
+                if (dst) {
+#pragma unroll
+                    for (int c = 0; c < D / 4; ++c)
+                        reinterpret_cast<float4 *>(dst)[c] =
+                            make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+                }
+            } else {
+                float gk[D];
+#pragma unroll
+                for (int d = 0; d < D; ++d) gk[d] = acc[d] * (kLn2 / sc);
+                float *dst = nullptr;
+                if (key < a.nc) {
+                    dst = a.dkc ? a.dkc + ((size_t)key * a.hkv + g) * D : nullptr;
+                } else {
+                    const int64_t nn = key - a.nc;
+                    float x[D];
+                    load_row_bf16<D>(a.k + ((size_t)nn * a.hkv + g) * D, x);
+                    qk_prologue_bwd<D>(x, gk, __ldg(a.pos + nn), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps);
+                    dst = a.dk + ((size_t)nn * a.hkv + g) * D;
+                }
+                if (dst) {
+#pragma unroll
+                    for (int c = 0; c < D / 4; ++c)
+                        reinterpret_cast<float4 *>(dst)[c] = make_float4(gk[4 * c], gk[4 * c + 1], gk[4 * c + 2], gk[4 * c + 3]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tbase, L::TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ dQ epilogue
+
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dq_kernel(DqArgs a) {
+    const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (row >= a.nq * a.hq) return;
+    const int64_t q = row / a.hq;
+    float g[D], x[D];
+    load_row_f32<D>(a.dq + (size_t)row * D, g);
+    const float sc = a.scale / ds_scale(a.bounds);
+#pragma unroll
+    for (int d = 0; d < D; ++d) g[d] *= sc;
+    load_row_bf16<D>(a.q + (size_t)row * D, x);
+    qk_prologue_bwd<D>(x, g, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps);
+    float4 *dst = reinterpret_cast<float4 *>(a.dq + (size_t)row * D);
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(g[4 * c], g[4 * c + 1], g[4 * c + 2], g[4 * c + 3]);
+}
+
+template <int D>
+int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
+    using L = BwdSmem<D>;
+    constexpr int DPAD = Geo<D>::DPAD;
+    uint8_t *ws = static_cast<uint8_t *>(io.workspace);
+    const size_t kvb = kv_image_bytes(P);
+    const size_t qb = q_image_bytes(P);
+    const size_t vb = q_vector_bytes(P);
+    auto *kimg16 = reinterpret_cast<__half *>(ws);
+    auto *vimg = reinterpret_cast<__nv_bfloat16 *>(ws + kvb);
+    auto *qimg16 = reinterpret_cast<__half *>(ws + 2 * kvb);
+    auto *doimg = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * kvb + qb);
+    auto *lse2 = reinterpret_cast<float *>(ws + 2 * kvb + 2 * qb);
+    auto *dsum = reinterpret_cast<float *>(ws + 2 * kvb + 2 * qb + vb);
+    auto *bounds = reinterpret_cast<float *>(ws + 2 * kvb + 2 * qb + 2 * vb);
+    if (cudaMemsetAsync(bounds, 0, 2 * sizeof(float), stream) != cudaSuccess) return BCA_ERR_CUDA;
+
+    PrepArgs pa;
+    pa.q = static_cast<const __nv_bfloat16 *>(io.q);
+    pa.dout = static_cast<const __nv_bfloat16 *>(io.dout);
+    pa.o = io.o;
+    pa.o_fp32 = (P.flags & BCA_O_FP32) ? 1 : 0;
+    pa.lse = io.lse;
+    pa.q_gain = io.q_gain;
+    pa.pos = P.d_pos;
+    pa.rope = P.d_rope;
+    pa.off0 = P.rope_axis_off[0];
+    pa.off1 = P.rope_axis_off[1];
+    pa.off2 = P.rope_axis_off[2];
+    pa.nq = P.nq;
+    pa.nqt = P.nqt;
+    pa.hq = P.hq;
+    pa.eps = P.eps;
+    pa.qscale = kLog2e / sqrtf((float)D);
+    pa.qimg16 = qimg16;
+    pa.doimg = doimg;
+    pa.bounds = bounds;
+    pa.lse2 = lse2;
+    pa.dsum = dsum;
+    pa.dq = io.dq;
+    {
+        ProfScope ps(P, BCA_KERNEL_BWD_PREP, stream);
+        bwd_prep_kernel<D><<<dim3((unsigned)P.nqt, (unsigned)P.hq), 128, 0, stream>>>(pa);
+    }
+    if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
+
+    BwdKVArgs ka;
+    ka.k = static_cast<const __nv_bfloat16 *>(io.k);
+    ka.v = static_cast<const __nv_bfloat16 *>(io.v);
+    ka.kc = static_cast<const __nv_bfloat16 *>(io.k_cache);
+    ka.vc = static_cast<const __nv_bfloat16 *>(io.v_cache);
+    ka.k_gain = io.k_gain;
+    ka.pos = P.d_pos;
+    ka.rope = P.d_rope;
+    ka.off0 = P.rope_axis_off[0];
+    ka.off1 = P.rope_axis_off[1];
+    ka.off2 = P.rope_axis_off[2];
+    ka.nc = P.nc;
+    ka.nk = P.nk;
+    ka.nkt = P.nkt;
+    ka.hkv = P.hkv;
+    ka.eps = P.eps;
+    ka.kimg16 = kimg16;
+    ka.vimg = vimg;
+    ka.bounds = bounds;
+    {
+        ProfScope ps(P, BCA_KERNEL_BWD_KV_IMAGE, stream);
+        bwd_kv_image_kernel<D><<<dim3((unsigned)P.nkt, (unsigned)P.hkv), 128, 0, stream>>>(ka);
+    }
+    if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
+
+    BwdArgs ba;
+    ba.kimg16 = kimg16;
+    ba.vimg = vimg;
+    ba.qimg16 = qimg16;
+    ba.doimg = doimg;
+    ba.bounds = bounds;
+    ba.lse2 = lse2;
+    ba.dsum = dsum;
+    ba.col_off = P.d_col_off;
+    ba.col_runs = P.d_col_runs;
+    ba.masks = P.d_masks;
+    ba.items = P.d_bwd_items;
+    ba.k = static_cast<const __nv_bfloat16 *>(io.k);
+    ba.k_gain = io.k_gain;
+    ba.pos = P.d_pos;
+    ba.rope = P.d_rope;
+    ba.off0 = P.rope_axis_off[0];
+    ba.off1 = P.rope_axis_off[1];
+    ba.off2 = P.rope_axis_off[2];
+    ba.nq = P.nq;
+    ba.nk = P.nk;
+    ba.nc = P.nc;
+    ba.nqt = P.nqt;
+    ba.nkt = P.nkt;
+    ba.hq = P.hq;
+    ba.hkv = P.hkv;
+    ba.eps = P.eps;
+    ba.dq = io.dq;
+    ba.dk = io.dk;
+    ba.dv = io.dv;
+    ba.dkc = io.dk_cache;
+    ba.dvc = io.dv_cache;
+    ba.status = P.d_status;
+    if (cudaFuncSetAttribute(bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES) != cudaSuccess)
+        return BCA_ERR_CUDA;
+    {
+        ProfScope ps(P, BCA_KERNEL_BWD, stream);
+        bwd_kernel<D><<<(unsigned)P.bwd_items.size(), 384, L::BYTES, stream>>>(ba);
+    }
+    if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
+
+    DqArgs da;
+    da.q = static_cast<const __nv_bfloat16 *>(io.q);
+    da.q_gain = io.q_gain;
+    da.pos = P.d_pos;
+    da.rope = P.d_rope;
+    da.off0 = P.rope_axis_off[0];
+    da.off1 = P.rope_axis_off[1];
+    da.off2 = P.rope_axis_off[2];
+    da.nq = P.nq;
+    da.hq = P.hq;
+    da.eps = P.eps;
+    da.scale = 1.0f / sqrtf((float)D);
+    da.dq = io.dq;
+    da.bounds = bounds;
+    {
+        ProfScope ps(P, BCA_KERNEL_BWD_DQ, stream);
+        const int64_t rows = P.nq * P.hq;
+        bwd_dq_kernel<D><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(da);
+    }
+    if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
+    (void)DPAD;
+    return BCA_OK;
+}
+
+}  // namespace
+
+size_t q_image_bytes(const Plan &P) {
+    const size_t b = (size_t)P.hq * (size_t)P.nqt * 128 * (size_t)P.dpad * 2;
+    return (b + 255) / 256 * 256;
+}
+
+size_t q_vector_bytes(const Plan &P) {
+    const size_t b = (size_t)P.hq * (size_t)P.nqt * 128 * 4;
+    return (b + 255) / 256 * 256;
+}
+
+size_t bwd_workspace_bytes(const Plan &P) {
+    return 2 * kv_image_bytes(P) + 2 * q_image_bytes(P) + 2 * q_vector_bytes(P) + 256;
+}
+
+int launch_bwd(Plan &P, const BwdIO &io, cudaStream_t stream) {
+    if (P.nq == 0 && P.nk == 0) return BCA_OK;
+    switch (P.d) {
+        case 24: return launch_bwd_d<24>(P, io, stream);
+        case 32: return launch_bwd_d<32>(P, io, stream);
+        case 48: return launch_bwd_d<48>(P, io, stream);
+        default: return BCA_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace bca

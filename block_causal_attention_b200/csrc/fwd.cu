@@ -25,6 +25,7 @@
 #include <cstdint>
 
 #include "kernels.hpp"
+#include "prologue.cuh"
 #include "sm100.cuh"
 
 namespace bca {
@@ -34,13 +35,6 @@ using namespace sm100;
 namespace {
 
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait; a healthy wait is microseconds
-
-template <int D>
-struct Geo {
-    static constexpr int DPAD = (D + 15) / 16 * 16;     // MMA k-granule for bf16 is 16
-    static constexpr int PAIRS = (D / 2) / 3;           // RoPE pairs per axis
-    static constexpr int TILE_BYTES = 128 * DPAD * 2;   // one K-hat or V tile image
-};
 
 struct KVArgs {
     const __nv_bfloat16 *k, *v, *kc, *vc;
@@ -75,67 +69,6 @@ struct FwdArgs {
     float *lse;
     int *status;
 };
-
-// ------------------------------------------------------------------ prologue math
-
-// RMS QK-Norm with gain, 3D RoPE at the packed position, then a scale; in place.
-template <int D>
-__device__ __forceinline__ void qk_prologue(float (&x)[D], uint32_t pos, const float *gain, const float *rope,
-                                            int32_t off0, int32_t off1, int32_t off2, float eps, float scale) {
-    constexpr int P = Geo<D>::PAIRS;
-    float ss = 0.f;
-#pragma unroll
-    for (int d = 0; d < D; ++d) ss = fmaf(x[d], x[d], ss);
-    const float r = rsqrtf(ss * (1.0f / D) + eps);
-#pragma unroll
-    for (int d = 0; d < D; ++d) x[d] = x[d] * r * (gain ? __ldg(gain + d) : 1.0f);
-    const int32_t p[3] = {(int32_t)(pos >> 16), (int32_t)((pos >> 8) & 255u), (int32_t)(pos & 255u)};
-    const int32_t off[3] = {off0, off1, off2};
-#pragma unroll
-    for (int a = 0; a < 3; ++a) {
-        const float2 *tab = reinterpret_cast<const float2 *>(rope) + (size_t)(off[a] + p[a]) * P;
-#pragma unroll
-        for (int k = 0; k < P; ++k) {
-            const float2 cs = __ldg(tab + k);
-            const int c0 = 2 * P * a + 2 * k;
-            const float y0 = x[c0], y1 = x[c0 + 1];
-            x[c0] = y0 * cs.x - y1 * cs.y;
-            x[c0 + 1] = y0 * cs.y + y1 * cs.x;
-        }
-    }
-#pragma unroll
-    for (int d = 0; d < D; ++d) x[d] *= scale;
-}
-
-template <int D>
-__device__ __forceinline__ void load_row_bf16(const __nv_bfloat16 *src, float (&x)[D]) {
-    const uint4 *s = reinterpret_cast<const uint4 *>(src);
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-        uint4 u = __ldg(s + c);
-        const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float2 f = __bfloat1622float2(b[e]);
-            x[c * 8 + 2 * e] = f.x;
-            x[c * 8 + 2 * e + 1] = f.y;
-        }
-    }
-}
-
-// Pack values [8c, 8c+8) of x (zero past D) into one 16-byte chunk of fp16.
-template <int D>
-__device__ __forceinline__ uint4 pack_chunk_f16(const float (&x)[D], int c) {
-    uint32_t w[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const int d0 = c * 8 + 2 * e;
-        const float lo = d0 < D ? x[d0] : 0.f;
-        const float hi = d0 + 1 < D ? x[d0 + 1] : 0.f;
-        w[e] = pack_f16x2(lo, hi);
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-}
 
 // ------------------------------------------------------------------ K-hat / V images
 

@@ -18,9 +18,24 @@ struct FwdIO {
     void *workspace;
 };
 
+struct BwdIO {
+    const void *q, *k, *v, *k_cache, *v_cache;
+    const float *q_gain, *k_gain;
+    const void *o;
+    const float *lse;
+    const void *dout;
+    float *dq, *dk, *dv, *dk_cache, *dv_cache;
+    void *workspace;
+};
+
 // Bytes of each K-hat / V image (all KV heads, all k-tiles), 256-byte rounded.
 size_t kv_image_bytes(const Plan &plan);
 size_t fwd_workspace_bytes(const Plan &plan);
+// Bytes of each Q-hat / dO image (all query heads, all q-tiles) and of each padded
+// per-query vector (LSE, Dsum); and the whole backward workspace.
+size_t q_image_bytes(const Plan &plan);
+size_t q_vector_bytes(const Plan &plan);
+size_t bwd_workspace_bytes(const Plan &plan);
 
 // Bracket a launch with events when the plan is profiling (no-op otherwise).
 struct ProfScope {
@@ -34,5 +49,7 @@ struct ProfScope {
 
 // Enqueue the forward on `stream`.  Returns BCA_OK or BCA_ERR_CUDA.
 int launch_fwd(Plan &plan, const FwdIO &io, cudaStream_t stream);
+// Enqueue the backward on `stream`.
+int launch_bwd(Plan &plan, const BwdIO &io, cudaStream_t stream);
 
 }  // namespace bca

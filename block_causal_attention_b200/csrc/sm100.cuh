@@ -138,6 +138,13 @@ __host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, uint32_t ab_fo
 }
 constexpr uint32_t kFmtF16 = 0, kFmtBF16 = 1;
 
+// Same with an operand's major-ness chosen: a_mn / b_mn = 1 marks that operand
+// MN-major (its 16-byte core-matrix rows run along M resp. N instead of K).
+__host__ __device__ constexpr uint32_t idesc_f32acc_major(int M, int N, uint32_t ab_format, uint32_t a_mn,
+                                                          uint32_t b_mn) {
+    return idesc_f32acc(M, N, ab_format) | (a_mn << 15) | (b_mn << 16);
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T (kind::f16: fp16 or bf16 operands), issued by one thread.
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t accumulate) {
@@ -180,6 +187,12 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
           "=r"(r[15])
         : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {

@@ -176,13 +176,30 @@ int bca_fwd_static_workspace(bca_plan_t plan, const void *q, const void *k, cons
                              const void *k_cache, const void *v_cache, const float *q_gain,
                              const float *k_gain, void *o, float *lse, void *stream);
 
+/* Backward.  Same q ... k_gain as bca_fwd; o and lse: the forward's outputs; dout:
+ * bf16 [Nq][Hq][D] upstream gradient of O.  Outputs (fp32): dq [Nq][Hq][D],
+ * dk, dv [Nq][Hkv][D] (new tokens, through QK-Norm and RoPE), dk_cache, dv_cache
+ * [Nc][Hkv][D] (cache keys are used as given, so their gradient is taken at the
+ * rotated keys; NULL = not wanted).  workspace: bca_workspace_bytes(BWD) bytes.
+ * dk, dv, dk_cache and dv_cache are reduced in a fixed order (bit-reproducible run to
+ * run); dq is accumulated with atomics, so its last bits may vary between runs. */
+int bca_bwd(bca_plan_t plan, const void *q, const void *k, const void *v,
+            const void *k_cache, const void *v_cache, const float *q_gain,
+            const float *k_gain, const void *o, const float *lse, const void *dout,
+            float *dq, float *dk, float *dv, float *dk_cache, float *dv_cache,
+            void *workspace, void *stream);
+
 /* Kernel kinds for per-kernel timing */
-#define BCA_KERNEL_KV_IMAGE 0  /* K-hat prologue + K/V tile images */
-#define BCA_KERNEL_FWD 1       /* attention forward */
-#define BCA_KERNEL_COUNT 2
+#define BCA_KERNEL_KV_IMAGE 0      /* K-hat prologue + K/V tile images */
+#define BCA_KERNEL_FWD 1           /* attention forward */
+#define BCA_KERNEL_BWD_PREP 2      /* Q-hat / dO images, LSE, Dsum */
+#define BCA_KERNEL_BWD_KV_IMAGE 3  /* K-hat / V images for the backward */
+#define BCA_KERNEL_BWD 4           /* attention backward */
+#define BCA_KERNEL_BWD_DQ 5        /* dQ prologue backward */
+#define BCA_KERNEL_COUNT 6
 
 /* Per-kernel device timing, a tracing aid.  While enabled (enable != 0), every
- * kernel that bca_fwd launches for this plan is bracketed by two CUDA events
+ * kernel that bca_fwd or bca_bwd launches for this plan is bracketed by two CUDA events
  * recorded on its stream.  bca_profile_read waits for those events and returns, for
  * one kernel kind, the number of launches and their summed device time in ms since
  * the last read (or enable), then forgets them.  Disabled by default. */

@@ -262,3 +262,17 @@ def backward(q, k, v, k_cache, v_cache, do, videos, slices, hq, hkv,
     dq = prologue_bwd(q, pos, dqh, base, eps, q_gain)
     dk = prologue_bwd(k, pos, dkh[nc:], base, eps, k_gain)
     return dq, dk, dvv[nc:], (dkh[:nc] if nc else None), (dvv[:nc] if nc else None), O, lse
+
+
+def backward_rows(q_rows, rows, k, v, k_cache, v_cache, do_rows, videos, slices, hq, hkv,
+                  base=(1e4, 1e4, 1e4), eps=1e-6, q_gain=None, k_gain=None):
+    """dq (w.r.t. the raw queries, through the prologue) for the listed query rows only;
+    q_rows / do_rows hold those rows' raw queries and upstream gradients."""
+    pos = positions(videos)
+    rows = np.asarray(rows, dtype=np.int64)
+    kh = full_keys(prologue(k, pos, base, eps, k_gain), k_cache)
+    vv = full_keys(v, v_cache)
+    qr = _f64(q_rows)
+    qh = prologue(qr, pos[rows], base, eps, q_gain)
+    dqh, O, lse = attn_bwd_rows(qh, rows, kh, vv, do_rows, slices, hq, hkv)
+    return prologue_bwd(qr, pos[rows], dqh, base, eps, q_gain)
