@@ -26,8 +26,9 @@ class Plan:
 
     def __init__(self, hq: int, hkv: int, d: int, videos, num_cache_keys: int = 0, slices=None,
                  rope_base=(1e4, 1e4, 1e4), eps: float = 1e-6, o_fp32: bool = False,
-                 host_only: bool = False):
-        flags = (_abi.BCA_O_FP32 if o_fp32 else 0) | (_abi.BCA_PLAN_HOST_ONLY if host_only else 0)
+                 host_only: bool = False, test_force_timeout: bool = False):
+        flags = (_abi.BCA_O_FP32 if o_fp32 else 0) | (_abi.BCA_PLAN_HOST_ONLY if host_only else 0) | \
+            (_abi.BCA_TEST_FORCE_TIMEOUT if test_force_timeout else 0)
         prob, keep = _abi.make_problem(hq, hkv, d, videos, num_cache_keys, slices, rope_base, eps, flags)
         self._lib = _abi.lib()
         self._h = _abi.ctypes.c_void_p()

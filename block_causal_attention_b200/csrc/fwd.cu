@@ -68,6 +68,8 @@ struct FwdArgs {
     void *o;
     float *lse;
     int *status;
+    uint64_t timeout_ns;  // per wait
+    int skip_loads;       // failure-detection test: issue no K/V loads
 };
 
 // ------------------------------------------------------------------ K-hat / V images
@@ -187,9 +189,10 @@ __device__ __forceinline__ void record_timeout(int *status, volatile int *abort_
     *abort_flag = 1;
 }
 
-__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, int *status, volatile int *abort_flag) {
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, int *status, volatile int *abort_flag,
+                                              uint64_t timeout_ns = kWaitTimeoutNs) {
     if (*abort_flag) return false;
-    if (mbar_wait(bar, parity, kWaitTimeoutNs)) return true;
+    if (mbar_wait(bar, parity, timeout_ns)) return true;
     record_timeout(status, abort_flag);
     return false;
 }
@@ -197,8 +200,8 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, int
 // Same, with the outcome made uniform across the warp (for warps that go on to
 // issue warp-collective tcgen05 loads/stores).
 __device__ __forceinline__ bool warp_wait_or_abort(uint32_t bar, uint32_t parity, int *status,
-                                                   volatile int *abort_flag) {
-    const bool ok = wait_or_abort(bar, parity, status, abort_flag);
+                                                   volatile int *abort_flag, uint64_t timeout_ns = kWaitTimeoutNs) {
+    const bool ok = wait_or_abort(bar, parity, status, abort_flag, timeout_ns);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -221,7 +224,7 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
     const Item item = a.items[blockIdx.x];
     const int64_t qt = item.q_tile;
     const int G = a.hq / a.hkv;
-    const int h0 = 2 * item.head_pair;
+    const int h0 = item.head0;
     const int g = h0 / G;
     const Run *rb = a.runs + a.run_off[qt];
     const Run *re = a.runs + a.run_off[qt + 1];
@@ -256,13 +259,13 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
 
     if (warp == 0) {
         // ------------------------------------------------ producer: K/V tiles
-        if (lane == 0 && n > 0) {
+        if (lane == 0 && n > 0 && !a.skip_loads) {
             int issued = 0;
             RunCursor cur(rb, re);
             for (int j = 0; j < n; ++j, cur.next()) {
                 const int stage = j % STAGES;
                 if (j >= STAGES &&
-                    !wait_or_abort(bar(L::B_KV_EMPTY + stage), ((j / STAGES) - 1) & 1, a.status, abort_flag))
+                    !wait_or_abort(bar(L::B_KV_EMPTY + stage), ((j / STAGES) - 1) & 1, a.status, abort_flag, a.timeout_ns))
                     break;
                 const size_t tile = ((size_t)g * a.nkt + cur.kt) * (128 * DPAD);
                 mbar_arrive_expect_tx(bar(L::B_KV_FULL + stage), 2 * L::TILE);
@@ -272,15 +275,15 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
             }
             // every issued copy must have landed before the CTA may exit
             for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
-                mbar_wait(bar(L::B_KV_FULL + j % STAGES), (j / STAGES) & 1, kWaitTimeoutNs);
+                mbar_wait(bar(L::B_KV_FULL + j % STAGES), (j / STAGES) & 1, a.timeout_ns);
         }
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0 && n > 0) {
-            bool ok = wait_or_abort(bar(L::B_Q_READY + 0), 0, a.status, abort_flag) &&
-                      wait_or_abort(bar(L::B_Q_READY + 1), 0, a.status, abort_flag) &&
-                      wait_or_abort(bar(L::B_KV_FULL + 0), 0, a.status, abort_flag);
+            bool ok = wait_or_abort(bar(L::B_Q_READY + 0), 0, a.status, abort_flag, a.timeout_ns) &&
+                      wait_or_abort(bar(L::B_Q_READY + 1), 0, a.status, abort_flag, a.timeout_ns) &&
+                      wait_or_abort(bar(L::B_KV_FULL + 0), 0, a.status, abort_flag, a.timeout_ns);
             tc_fence_after();
             auto issue_s = [&](int slot, int stage) {
                 const uint32_t qa = sbase + L::OFF_Q + slot * L::Q_BYTES;
@@ -313,18 +316,18 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
                     const bool more = j + 1 < n;
                     const int nstage = (j + 1) % STAGES;
                     if (more) {
-                        ok = wait_or_abort(bar(L::B_KV_FULL + nstage), ((j + 1) / STAGES) & 1, a.status, abort_flag);
+                        ok = wait_or_abort(bar(L::B_KV_FULL + nstage), ((j + 1) / STAGES) & 1, a.status, abort_flag, a.timeout_ns);
                         tc_fence_after();
                     }
                     for (int s = 0; s < 2 && ok; ++s) {
                         if (more) {
-                            ok = wait_or_abort(bar(L::B_S_FREE + s), j & 1, a.status, abort_flag);
+                            ok = wait_or_abort(bar(L::B_S_FREE + s), j & 1, a.status, abort_flag, a.timeout_ns);
                             if (!ok) break;
                             tc_fence_after();
                             issue_s(s, nstage);
                             mma_commit(bar(L::B_S_FULL + s));
                         }
-                        ok = wait_or_abort(bar(L::B_P_FULL + s), j & 1, a.status, abort_flag);
+                        ok = wait_or_abort(bar(L::B_P_FULL + s), j & 1, a.status, abort_flag, a.timeout_ns);
                         if (!ok) break;
                         tc_fence_after();
                         issue_pv(s, stage, j > 0);
@@ -335,7 +338,7 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
             }
             // all issued MMAs must be complete before TMEM is released
             mma_commit(bar(L::B_MMA_DONE));
-            mbar_wait(bar(L::B_MMA_DONE), 0, kWaitTimeoutNs);
+            mbar_wait(bar(L::B_MMA_DONE), 0, a.timeout_ns);
         }
         __syncwarp();
     } else if (warp >= 4) {
@@ -372,7 +375,7 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
         bool ok = true;
         RunCursor cur(rb, re);
         for (int j = 0; j < n; ++j, cur.next()) {
-            ok = warp_wait_or_abort(bar(L::B_S_FULL + slot), j & 1, a.status, abort_flag);
+            ok = warp_wait_or_abort(bar(L::B_S_FULL + slot), j & 1, a.status, abort_flag, a.timeout_ns);
             if (!ok) break;
             tc_fence_after();
             float s[128];
@@ -414,7 +417,7 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
             l = l * alpha + sum;
 
             if (j > 0) {
-                ok = warp_wait_or_abort(bar(L::B_O_DONE + slot), (j - 1) & 1, a.status, abort_flag);
+                ok = warp_wait_or_abort(bar(L::B_O_DONE + slot), (j - 1) & 1, a.status, abort_flag, a.timeout_ns);
                 if (!ok) break;
                 tc_fence_after();
                 if (__any_sync(0xffffffffu, rescale)) {
@@ -448,7 +451,7 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
 #pragma unroll
         for (int d = 0; d < DPAD; ++d) o[d] = 0.f;
         if (n > 0 && ok) {
-            ok = warp_wait_or_abort(bar(L::B_O_DONE + slot), (n - 1) & 1, a.status, abort_flag);
+            ok = warp_wait_or_abort(bar(L::B_O_DONE + slot), (n - 1) & 1, a.status, abort_flag, a.timeout_ns);
             tc_fence_after();
             if (ok) {
 #pragma unroll
@@ -546,6 +549,8 @@ int launch_fwd_d(Plan &P, const FwdIO &io, cudaStream_t stream) {
     fa.o = io.o;
     fa.lse = io.lse;
     fa.status = P.d_status;
+    fa.timeout_ns = (P.flags & BCA_TEST_FORCE_TIMEOUT) ? 1000000ull : kWaitTimeoutNs;
+    fa.skip_loads = (P.flags & BCA_TEST_FORCE_TIMEOUT) ? 1 : 0;
     if (cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES) != cudaSuccess)
         return BCA_ERR_CUDA;
     {

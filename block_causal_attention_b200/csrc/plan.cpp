@@ -121,7 +121,7 @@ void compile_q_tile(const Plan &P, int64_t qt, TileOut &out) {
 
 int validate_problem(const bca_problem *p, Plan &P) {
     if (!p) return BCA_ERR_INVALID_ARGUMENT;
-    if (p->flags & ~(BCA_O_FP32 | BCA_PLAN_HOST_ONLY)) return BCA_ERR_INVALID_ARGUMENT;
+    if (p->flags & ~(BCA_O_FP32 | BCA_PLAN_HOST_ONLY | BCA_TEST_FORCE_TIMEOUT)) return BCA_ERR_INVALID_ARGUMENT;
     if (p->num_q_heads <= 0 || p->num_kv_heads <= 0) return BCA_ERR_INVALID_ARGUMENT;
     if (p->num_q_heads % p->num_kv_heads != 0) return BCA_ERR_UNSUPPORTED;
     if ((p->num_q_heads / p->num_kv_heads) % 2 != 0) return BCA_ERR_UNSUPPORTED;
@@ -272,18 +272,20 @@ int compile_plan(Plan &P) {
 
     // ---- items, longest first; ties grouped by KV group then q-tile so that CTAs
     //      running together stream the same K/V tiles ----
-    const int npairs = P.hq / 2, G = P.hq / P.hkv;
+    const int G = P.hq / P.hkv;
+    P.heads_per_item = 2;
+    const int nsets = P.hq / P.heads_per_item;
     P.items.clear();
-    P.items.reserve((size_t)P.nqt * npairs);
+    P.items.reserve((size_t)P.nqt * nsets);
     for (int64_t qt = 0; qt < P.nqt; ++qt)
-        for (int hp = 0; hp < npairs; ++hp) P.items.push_back({(int32_t)qt, hp});
+        for (int hs = 0; hs < nsets; ++hs) P.items.push_back({(int32_t)qt, hs * P.heads_per_item});
     std::stable_sort(P.items.begin(), P.items.end(), [&](const Item &x, const Item &y) {
         const int32_t cx = P.qt_tiles[x.q_tile], cy = P.qt_tiles[y.q_tile];
         if (cx != cy) return cx > cy;
-        const int gx = 2 * x.head_pair / G, gy = 2 * y.head_pair / G;
+        const int gx = x.head0 / G, gy = y.head0 / G;
         if (gx != gy) return gx < gy;
         if (x.q_tile != y.q_tile) return x.q_tile < y.q_tile;
-        return x.head_pair < y.head_pair;
+        return x.head0 < y.head0;
     });
 
     // ---- positions and RoPE tables ----

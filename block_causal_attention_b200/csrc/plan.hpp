@@ -19,15 +19,16 @@ struct Run {
     int32_t kt_begin, kt_end, mask_idx, pad;
 };
 
-// Forward work item: q-tile x pair of query heads (2*head_pair, 2*head_pair+1),
-// both in the same KV group so they stream the same K/V tiles.
+// Forward work item: q-tile x a set of heads_per_item query heads starting at
+// head0, all in one KV group so they stream the same K/V tiles.
 struct Item {
-    int32_t q_tile, head_pair;
+    int32_t q_tile, head0;
 };
 
 struct Plan {
     // problem
     int hq = 0, hkv = 0, d = 0, dpad = 0;
+    int heads_per_item = 2;  // query heads per forward CTA: 4 when the group size allows
     int64_t nq = 0, nk = 0, nc = 0;
     uint32_t flags = 0;
     float base[3] = {1e4f, 1e4f, 1e4f};

@@ -72,6 +72,9 @@ extern "C" {
 /* bca_problem.flags */
 #define BCA_O_FP32 0x1u          /* write O as fp32 instead of bf16 */
 #define BCA_PLAN_HOST_ONLY 0x2u  /* compile the mask on the host only (no CUDA calls) */
+#define BCA_TEST_FORCE_TIMEOUT 0x4u /* failure-detection test: bca_fwd's K/V loads are not
+                                       issued and its waits give up after 1 ms, so every
+                                       CTA records BCA_ERR_DEVICE_TIMEOUT and exits cleanly */
 
 /* bca_workspace_bytes(pass) */
 #define BCA_PASS_FWD 0
@@ -102,7 +105,7 @@ typedef struct {
                                    every chunk of the first video */
     float rope_base[3];         /* RoPE base per axis (t, h, w) */
     float norm_eps;             /* QK-Norm epsilon */
-    uint32_t flags;             /* BCA_O_FP32 | BCA_PLAN_HOST_ONLY */
+    uint32_t flags;             /* BCA_O_FP32 | BCA_PLAN_HOST_ONLY | BCA_TEST_FORCE_TIMEOUT */
 } bca_problem;
 
 typedef struct bca_plan_s *bca_plan_t;
@@ -113,7 +116,7 @@ typedef struct {
     int64_t num_q_tiles, num_k_tiles;
     int64_t num_runs;            /* runs of consecutive k-tiles over all q-tiles */
     int64_t num_full_tiles, num_partial_tiles;
-    int64_t num_items;           /* forward work items (q-tile x head pair) */
+    int64_t num_items;           /* forward work items (q-tile x 2 or 4 heads of a group) */
     int64_t visible_pairs;       /* visible (query, key) pairs per head */
     int32_t head_dim_padded;     /* D rounded up to the MMA k-granule (16) */
     int32_t tile_q, tile_k;

@@ -121,7 +121,7 @@ def test_tile_classes_of_720p_pipelined():
     tiles = inf["num_full_tiles"] + inf["num_partial_tiles"]
     # every visible pair lies in a compiled tile and partial tiles are rare
     assert inf["num_partial_tiles"] < 0.001 * tiles
-    assert inf["num_items"] == 675 * 64
+    assert inf["num_items"] == 675 * 64  # 2 query heads per item
 
 
 # ---------------------------------------------------------------- argument checks
