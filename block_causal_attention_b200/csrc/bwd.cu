@@ -4,7 +4,7 @@
 //                        log2(e)/sqrt(D)) as an fp16 image, bit-identical to the forward's
 //                        Q tile, so S and hence P are recomputed exactly as the forward saw
 //                        them; dO as a bf16 image; LSE in log2 units; Dsum_i = dO_i . O_i;
-//                        the largest |dO_i|; zeroes the dQ rows.
+//                        the largest |dO_i|.
 //   bwd_kv_image_kernel: K-hat (fp16, as in the forward) and V (bf16) images in the
 //                        key-row core layout, and the largest |v_j|.
 //   Precision: dP^T = V dO^T and dV = P^T dO run on bf16 (exact inputs; P rounded to
@@ -16,11 +16,16 @@
 //                        (query tile, query head of the group) that sees the key tile, in
 //                        a fixed order, so dK and dV are accumulated deterministically
 //                        in tensor memory.  Per step it recomputes S^T = K Q^T and
-//                        dP^T = V dO^T, forms P^T = exp2(S^T - LSE) and
-//                        dS^T = P^T (dP^T - Dsum) in the compute warps, then issues
-//                        dV += P^T dO, dK += dS^T Q and dQ_part = dS K; dQ_part is added
-//                        to dQ with float4 atomics (the one non-deterministic sum).
-//   bwd_dq_kernel      : dQ <- prologue backward (RoPE^T, RMS-norm^T) of dQ-hat, in place.
+//                        dP^T = V dO^T, forms P^T = exp2(S^T - LSE) (bf16, into tensor
+//                        memory) and dS^T = P^T (dP^T - Dsum) (fp16, into shared memory)
+//                        in the compute warps, then issues dV += P^T dO (A operand from
+//                        tensor memory), dK += dS^T Q and dQ_part = dS K.  Each compute
+//                        warp adds its 32 x Dpad/2 block of dQ_part to an fp32 accumulator
+//                        with one bulk reduce-add of the TMA engine (the one
+//                        non-deterministic sum); the accumulator keeps each (head, query
+//                        tile) block contiguous so no per-row atomics go through L1.
+//   bwd_dq_kernel      : dQ <- prologue backward (RoPE^T, RMS-norm^T) of the accumulated
+//                        dQ-hat.
 //
 // Gradients of the forward defined in fwd.cu; the pages give the forward only
 // (MAGI-1 research notes (zhao9797.github.io), "Infra > MagiAttention >
@@ -58,7 +63,7 @@ struct PrepArgs {
     float eps, qscale;
     __half *qimg16;
     __nv_bfloat16 *doimg;
-    float *lse2, *dsum, *dq;
+    float *lse2, *dsum;
     float *bounds;  // [0] = max |dO_i| (atomic max on the float bits)
 };
 
@@ -93,7 +98,8 @@ struct BwdArgs {
     int64_t nq, nk, nc, nqt, nkt;
     int hq, hkv;
     float eps;
-    float *dq, *dk, *dv, *dkc, *dvc;
+    float *dqacc;  // fp32 dQ-hat accumulator, [Hq][query tile][2][128][DPAD / 2]
+    float *dk, *dv, *dkc, *dvc;
     int *status;
 };
 
@@ -103,10 +109,11 @@ struct DqArgs {
     const uint32_t *pos;
     const float *rope;
     int32_t off0, off1, off2;
-    int64_t nq;
+    int64_t nq, nqt;
     int hq;
     float eps, scale;
     const float *bounds;
+    const float *dqacc;
     float *dq;
 };
 
@@ -194,9 +201,6 @@ __global__ void __launch_bounds__(128) bwd_prep_kernel(PrepArgs a) {
         for (int d = 0; d < D; ++d) dsum = fmaf(g[d], x[d], dsum);
         const float L = a.lse[(size_t)h * a.nq + q];
         if (L > -INFINITY) lse2 = L * kLog2e;  // a row with no visible key keeps +inf: P = 0
-        float4 *dqr = reinterpret_cast<float4 *>(a.dq + row);
-#pragma unroll
-        for (int c = 0; c < D / 4; ++c) dqr[c] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     a.lse2[((size_t)h * a.nqt + qt) * 128 + t] = lse2;
     a.dsum[((size_t)h * a.nqt + qt) * 128 + t] = dsum;
@@ -249,24 +253,35 @@ __global__ void __launch_bounds__(128) bwd_kv_image_kernel(BwdKVArgs a) {
 template <int D>
 struct BwdSmem {
     static constexpr int DPAD = Geo<D>::DPAD;
+    static constexpr int HALF = DPAD / 2;  // dQ columns per compute warpgroup
     static constexpr int TILE = 128 * DPAD * 2;
-    static constexpr int STAGES = 2;
+    static constexpr int STAGES = 4;
     static constexpr int OFF_K16 = 0;
     static constexpr int OFF_V = TILE;
     static constexpr int OFF_STAGE = 2 * TILE;
     static constexpr int ST_Q16 = 0, ST_DO = TILE, ST_LSE = 2 * TILE, ST_DSUM = 2 * TILE + 512,
                          ST_MASK = 2 * TILE + 1024;
     static constexpr int STAGE_BYTES = 2 * TILE + 1024 + 2048;
-    static constexpr int OFF_PT = OFF_STAGE + STAGES * STAGE_BYTES;  // P^T, bf16 128x128
-    static constexpr int OFF_DST = OFF_PT + 32768;                    // dS^T, fp16 128x128
-    static constexpr int OFF_BAR = OFF_DST + 32768;
-    static constexpr int B_KV = 0, B_ST_FULL = 1, B_ST_EMPTY = 3, B_S_FULL = 5, B_S_FREE = 6, B_DS_READY = 7,
-                         B_PDS_FREE = 8, B_DQ_FULL = 9, B_DQ_FREE = 10, B_MMA_DONE = 11, NBAR = 12;
+    // dS^T (fp16 128x128), double-buffered by item parity so the compute warps write
+    // item i+1 while the dK / dQ MMAs of item i still read item i
+    static constexpr int OFF_DST = OFF_STAGE + STAGES * STAGE_BYTES;  // [2]
+    // dQ_part staging for the bulk reduce: one 32-row x HALF block per compute warp
+    static constexpr int WARP_STAGE = 32 * HALF * 4;
+    static constexpr int OFF_DQS = OFF_DST + 2 * 32768;  // [8]
+    static constexpr int OFF_BAR = OFF_DQS + 8 * WARP_STAGE;
+    static constexpr int B_KV = 0, B_ST_FULL = 1, B_ST_EMPTY = 1 + STAGES, B_S_FULL = 1 + 2 * STAGES,
+                         B_S_FREE = B_S_FULL + 1, B_DS_READY = B_S_FULL + 2, B_PT_FREE = B_S_FULL + 3,
+                         B_DS_FREE = B_S_FULL + 4 /* [2] */, B_DQ_FULL = B_S_FULL + 6, B_DQ_FREE = B_S_FULL + 7,
+                         B_MMA_DONE = B_S_FULL + 8, NBAR = B_S_FULL + 9;
     static constexpr int OFF_TMEM_PTR = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ABORT = OFF_TMEM_PTR + 4;
     static constexpr int BYTES = OFF_ABORT + 12;
+    static_assert(BYTES <= 232448, "shared memory");
+    // tensor memory: S^T and dP^T (fp32, 128 columns each), P^T (bf16 pairs, 64 columns,
+    // the A operand of dV), then dQ_part, dV and dK (fp32, DPAD <= 64 columns each)
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 256, COL_DV = 320, COL_DK = 384;
+    static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_PT = 256, COL_DQ = 320, COL_DV = 384, COL_DK = 448;
+    static_assert(DPAD <= 64, "tensor memory map");
 };
 
 // Walks (query tile, query head) items of one key tile: runs of query tiles, and
@@ -305,10 +320,11 @@ template <int D>
 __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
     using L = BwdSmem<D>;
     constexpr int DPAD = L::DPAD;
+    constexpr int HALF = L::HALF;
     constexpr int STAGES = L::STAGES;
     constexpr uint32_t IDESC_S = idesc_f32acc(128, 128, kFmtF16);     // S^T: fp16 K-hat, Q-hat
     constexpr uint32_t IDESC_DP = idesc_f32acc(128, 128, kFmtBF16);   // dP^T: bf16 V, dO
-    constexpr uint32_t IDESC_DV = idesc_f32acc_major(128, DPAD, kFmtBF16, 0, 1);  // dV: B MN-major
+    constexpr uint32_t IDESC_DV = idesc_f32acc_major(128, DPAD, kFmtBF16, 0, 1);  // dV: A in TMEM, B MN-major
     constexpr uint32_t IDESC_DK = idesc_f32acc_major(128, DPAD, kFmtF16, 0, 1);   // dK: B MN-major
     constexpr uint32_t IDESC_DQ = idesc_f32acc_major(128, DPAD, kFmtF16, 1, 1);   // dQ: A and B MN-major
 
@@ -338,7 +354,9 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
         mbar_init(bar(L::B_S_FULL), 1);
         mbar_init(bar(L::B_S_FREE), 256);
         mbar_init(bar(L::B_DS_READY), 256);
-        mbar_init(bar(L::B_PDS_FREE), 1);
+        mbar_init(bar(L::B_PT_FREE), 1);
+        mbar_init(bar(L::B_DS_FREE), 1);
+        mbar_init(bar(L::B_DS_FREE + 1), 1);
         mbar_init(bar(L::B_DQ_FULL), 1);
         mbar_init(bar(L::B_DQ_FREE), 256);
         mbar_init(bar(L::B_MMA_DONE), 1);
@@ -381,16 +399,19 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                 if (mk >= 0) bulk_g2s(st + L::ST_MASK, a.masks + (size_t)mk * 512, 2048, bar(L::B_ST_FULL + s));
                 ++issued;
             }
-            mbar_wait(bar(L::B_KV), 0, kWaitTimeoutNs);
-            for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
-                mbar_wait(bar(L::B_ST_FULL + i % STAGES), (i / STAGES) & 1, kWaitTimeoutNs);
+            // every issued copy must have landed before the CTA may exit (matters when
+            // the consumers stopped early)
+            for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+                if (!mbar_wait(bar(L::B_ST_FULL + j % STAGES), (j / STAGES) & 1, kWaitTimeoutNs))
+                    atomicOr(a.status, kStatusTimeout);
+            if (!mbar_wait(bar(L::B_KV), 0, kWaitTimeoutNs)) atomicOr(a.status, kStatusTimeout);
         }
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t k16 = sbase + L::OFF_K16, vb = sbase + L::OFF_V;
-            const uint32_t pt = sbase + L::OFF_PT, dst = sbase + L::OFF_DST;
+            const uint32_t dst0 = sbase + L::OFF_DST;
             auto stage = [&](int i) -> uint32_t { return sbase + L::OFF_STAGE + (i % STAGES) * L::STAGE_BYTES; };
             // S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 128 queries, K = DPAD; all K-major)
             auto issue_s_dp = [&](int i) {
@@ -422,20 +443,25 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                     issue_s_dp(i + 1);
                     mma_commit(bar(L::B_S_FULL));
                 }
+                const int b = i & 1;
+                const uint32_t dst = dst0 + b * 32768;
                 ok = wait_abort(bar(L::B_DS_READY), i & 1, a.status, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                // dV += P^T dO and dK += dS^T Q (M = 128 keys, N = DPAD, K = 128 queries):
-                // A K-major from P^T / dS^T, B MN-major from the dO / Q image
+                // dV += P^T dO (M = 128 keys, N = DPAD, K = 128 queries): A = P^T in tensor
+                // memory (16 queries per 8 columns), B MN-major from the dO image
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-                    mma_f16(tbase + L::COL_DV, smem_desc(pt + kk * 4096, 2048, 128),
-                            smem_desc(st + L::ST_DO + kk * 256, 128, 2048), IDESC_DV, acc);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16_ts(tbase + L::COL_DV, tbase + L::COL_PT + 8 * kk,
+                               smem_desc(st + L::ST_DO + kk * 256, 128, 2048), IDESC_DV, (i > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(bar(L::B_PT_FREE));
+                // dK += dS^T Q: A K-major from the dS^T buffer, B MN-major from the Q image
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
                     mma_f16(tbase + L::COL_DK, smem_desc(dst + kk * 4096, 2048, 128),
-                            smem_desc(st + L::ST_Q16 + kk * 256, 128, 2048), IDESC_DK, acc);
-                }
-                if (i > 0) {
+                            smem_desc(st + L::ST_Q16 + kk * 256, 128, 2048), IDESC_DK, (i > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(bar(L::B_ST_EMPTY + i % STAGES));
+                if (i > 0) {  // the compute warps have read dQ_part of item i - 1
                     ok = wait_abort(bar(L::B_DQ_FREE), (i - 1) & 1, a.status, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
@@ -447,11 +473,13 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                     mma_f16(tbase + L::COL_DQ, smem_desc(dst + kk * 256, 128, 2048),
                             smem_desc(k16 + kk * 256, 128, 2048), IDESC_DQ, kk > 0);
                 mma_commit(bar(L::B_DQ_FULL));
-                mma_commit(bar(L::B_ST_EMPTY + i % STAGES));
-                mma_commit(bar(L::B_PDS_FREE));
+                mma_commit(bar(L::B_DS_FREE + b));
             }
             mma_commit(bar(L::B_MMA_DONE));
-            mbar_wait(bar(L::B_MMA_DONE), 0, kWaitTimeoutNs);
+            if (!mbar_wait(bar(L::B_MMA_DONE), 0, kWaitTimeoutNs)) {
+                atomicOr(a.status, kStatusTimeout);
+                *abort_flag = 1;
+            }
         }
         __syncwarp();
     } else if (warp >= 4) {
@@ -461,35 +489,39 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
         const int r = quarter * 32 + lane;  // key row of S^T / dP^T; query row of dQ_part
         const int c0 = 64 * wg;             // this warpgroup's query columns
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        uint4 *ptb = reinterpret_cast<uint4 *>(smem + L::OFF_PT);
-        uint4 *dsb = reinterpret_cast<uint4 *>(smem + L::OFF_DST);
+        uint4 *dsb0 = reinterpret_cast<uint4 *>(smem + L::OFF_DST);
+        float *stage_dq = reinterpret_cast<float *>(smem + L::OFF_DQS + (warp - 4) * L::WARP_STAGE);
         bool ok = true;
         int prev_qt = 0, prev_h = 0;
         const float sc = ds_scale(a.bounds);
 
+        // dQ_part of item j: this warp's 32 rows x HALF columns leave tensor memory, are
+        // staged in shared memory and added to the fp32 accumulator tile by one bulk
+        // reduce (TMA engine); the tile of (head, query tile) is laid out
+        // [2 column halves][128 rows][HALF], so the block is contiguous
         auto dq_epilogue = [&](int j, int qt_j, int h_j) -> bool {
             if (!warp_wait_abort(bar(L::B_DQ_FULL), j & 1, a.status, abort_flag)) return false;
             tc_fence_after();
-            constexpr int HALF = DPAD / 2;
-            float v[HALF];
+            uint32_t v[HALF];
 #pragma unroll
-            for (int c = 0; c < HALF / 8; ++c) {
-                uint32_t r8[8];
-                tmem_ld8(tbase + lane_off + L::COL_DQ + wg * HALF + 8 * c, r8);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[8 * c + e] = __uint_as_float(r8[e]);
-            }
+            for (int c = 0; c < HALF / 8; ++c)
+                tmem_ld8(tbase + lane_off + L::COL_DQ + wg * HALF + 8 * c, *reinterpret_cast<uint32_t(*)[8]>(&v[8 * c]));
+            tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(bar(L::B_DQ_FREE));
-            const int64_t qrow = (int64_t)qt_j * 128 + r;
-            if (qrow < a.nq) {
-                float *dst = a.dq + ((size_t)qrow * a.hq + h_j) * D + wg * HALF;
+            if (lane == 0) bulk_wait_group_read0();  // the previous reduce has read the staging block
+            __syncwarp();
+            float4 *row = reinterpret_cast<float4 *>(stage_dq + lane * HALF);
 #pragma unroll
-                for (int c = 0; c < HALF / 4; ++c)
-                    if (wg * HALF + 4 * c < D)
-                        atomicAdd(reinterpret_cast<float4 *>(dst + 4 * c),
-                                  make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]));
+            for (int c = 0; c < HALF / 4; ++c)
+                row[c] = make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
+                                     __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3]));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                float *dst = a.dqacc + ((((size_t)h_j * a.nqt + qt_j) * 2 + wg) * 128 + 32 * quarter) * HALF;
+                bulk_reduce_add_f32(dst, smem_u32(stage_dq), L::WARP_STAGE);
+                bulk_commit_group();
             }
             return true;
         };
@@ -503,48 +535,62 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                  warp_wait_abort(bar(L::B_S_FULL), i & 1, a.status, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            float sv[64], dp[64];
-            {
-                uint32_t u[64];
-                tmem_ld32(tbase + lane_off + L::COL_S + c0, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-                tmem_ld32(tbase + lane_off + L::COL_S + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(u[c]);
-                tmem_ld32(tbase + lane_off + L::COL_DP + c0, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-                tmem_ld32(tbase + lane_off + L::COL_DP + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 64; ++c) dp[c] = __uint_as_float(u[c]);
-            }
+            uint32_t su[64], du[64];  // S^T and dP^T values of this thread's 64 columns (raw bits)
+            tmem_ld32(tbase + lane_off + L::COL_S + c0, *reinterpret_cast<uint32_t(*)[32]>(&su[0]));
+            tmem_ld32(tbase + lane_off + L::COL_S + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&su[32]));
+            tmem_ld32(tbase + lane_off + L::COL_DP + c0, *reinterpret_cast<uint32_t(*)[32]>(&du[0]));
+            tmem_ld32(tbase + lane_off + L::COL_DP + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&du[32]));
+            tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(bar(L::B_S_FREE));
 
-            const float *lse2 = reinterpret_cast<const float *>(st + L::ST_LSE) + c0;
-            const float *dsum = reinterpret_cast<const float *>(st + L::ST_DSUM) + c0;
+            const float4 *lse4 = reinterpret_cast<const float4 *>(st + L::ST_LSE) + c0 / 4;
+            const float4 *dsum4 = reinterpret_cast<const float4 *>(st + L::ST_DSUM) + c0 / 4;
             const bool partial = cur.r->mask_idx >= 0;
             const uint32_t *mask = reinterpret_cast<const uint32_t *>(st + L::ST_MASK);
-#pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                float p = ex2(sv[c] - lse2[c]);
-                if (partial && !((mask[(c0 + c) * 4 + r / 32] >> (r % 32)) & 1u)) p = 0.f;
-                sv[c] = p;
-                dp[c] = p * (dp[c] - dsum[c]) * sc;
-            }
-            if (i > 0) {
-                ok = warp_wait_abort(bar(L::B_PDS_FREE), (i - 1) & 1, a.status, abort_flag);
+            const int b = i & 1;
+            if (i > 1) {  // dS^T buffer b was last read by the dK / dQ MMAs of item i - 2
+                ok = warp_wait_abort(bar(L::B_DS_FREE + b), ((i >> 1) - 1) & 1, a.status, abort_flag);
                 if (!ok) break;
             }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int idx = img_chunk(c0 / 8 + k, r);
-                ptb[idx] = make_uint4(pack_bf16x2(sv[8 * k], sv[8 * k + 1]), pack_bf16x2(sv[8 * k + 2], sv[8 * k + 3]),
-                                      pack_bf16x2(sv[8 * k + 4], sv[8 * k + 5]),
-                                      pack_bf16x2(sv[8 * k + 6], sv[8 * k + 7]));
-                dsb[idx] = make_uint4(pack_f16x2(dp[8 * k], dp[8 * k + 1]), pack_f16x2(dp[8 * k + 2], dp[8 * k + 3]),
-                                      pack_f16x2(dp[8 * k + 4], dp[8 * k + 5]), pack_f16x2(dp[8 * k + 6], dp[8 * k + 7]));
+            if (i > 0) {  // the dV MMAs of item i - 1 have read P^T from tensor memory
+                ok = warp_wait_abort(bar(L::B_PT_FREE), (i - 1) & 1, a.status, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
             }
+            uint4 *dsb = dsb0 + b * 2048;
+            // P = exp2(S - LSE) and dS = P (dP - Dsum), 16 columns at a time: P as bf16
+            // pairs into tensor memory, dS as fp16 into the dS^T image
+#pragma unroll
+            for (int k2 = 0; k2 < 4; ++k2) {
+                uint32_t pw[8];
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int k = 2 * k2 + hf;
+                    const float4 l0 = lse4[2 * k], l1 = lse4[2 * k + 1], d0 = dsum4[2 * k], d1 = dsum4[2 * k + 1];
+                    const float lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+                    const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+                    uint32_t dw[4];
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        const int c = 8 * k + e;
+                        float p0 = ex2(__uint_as_float(su[c]) - lv[e]);
+                        float p1 = ex2(__uint_as_float(su[c + 1]) - lv[e + 1]);
+                        if (partial) {
+                            if (!((mask[(c0 + c) * 4 + r / 32] >> (r % 32)) & 1u)) p0 = 0.f;
+                            if (!((mask[(c0 + c + 1) * 4 + r / 32] >> (r % 32)) & 1u)) p1 = 0.f;
+                        }
+                        pw[4 * hf + e / 2] = pack_bf16x2(p0, p1);
+                        dw[e / 2] = pack_f16x2(p0 * (__uint_as_float(du[c]) - dv[e]) * sc,
+                                               p1 * (__uint_as_float(du[c + 1]) - dv[e + 1]) * sc);
+                    }
+                    dsb[img_chunk(c0 / 8 + k, r)] = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+                }
+                tmem_st8(tbase + lane_off + L::COL_PT + c0 / 2 + 8 * k2, pw);
+            }
+            tmem_wait_st();
             fence_proxy_async_smem();
+            tc_fence_before();
             mbar_arrive(bar(L::B_DS_READY));
             if (i > 0 && !dq_epilogue(i - 1, prev_qt, prev_h)) {
                 ok = false;
@@ -554,6 +600,7 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
             prev_h = h;
         }
         if (ok && n > 0) ok = dq_epilogue(n - 1, prev_qt, prev_h);
+        if (lane == 0) bulk_wait_group0();  // the reduces have landed and read their staging
 
         // dK / dV epilogue: warpgroup 0 writes dV, warpgroup 1 dK (through the
         // prologue backward for new keys)
@@ -616,19 +663,38 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
 
 // ------------------------------------------------------------------ dQ epilogue
 
+// one thread per (query, query head), queries fastest so the accumulator reads coalesce
 template <int D>
-__global__ void __launch_bounds__(256) bwd_dq_kernel(DqArgs a) {
-    const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (row >= a.nq * a.hq) return;
-    const int64_t q = row / a.hq;
+__global__ void __launch_bounds__(128) bwd_dq_kernel(DqArgs a) {
+    constexpr int HALF = Geo<D>::DPAD / 2;
+    const int64_t q = (int64_t)blockIdx.x * 128 + threadIdx.x;
+    const int h = blockIdx.y;
+    if (q >= a.nq) return;
+    const int64_t qt = q / 128;
+    const int rr = (int)(q % 128);
     float g[D], x[D];
-    load_row_f32<D>(a.dq + (size_t)row * D, g);
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        const float4 *src =
+            reinterpret_cast<const float4 *>(a.dqacc + ((((size_t)h * a.nqt + qt) * 2 + hf) * 128 + rr) * HALF);
+#pragma unroll
+        for (int c = 0; c < HALF / 4; ++c) {
+            if (hf * HALF + 4 * c < D) {
+                const float4 f = src[c];
+                g[hf * HALF + 4 * c] = f.x;
+                g[hf * HALF + 4 * c + 1] = f.y;
+                g[hf * HALF + 4 * c + 2] = f.z;
+                g[hf * HALF + 4 * c + 3] = f.w;
+            }
+        }
+    }
     const float sc = a.scale / ds_scale(a.bounds);
 #pragma unroll
     for (int d = 0; d < D; ++d) g[d] *= sc;
-    load_row_bf16<D>(a.q + (size_t)row * D, x);
+    const size_t row = (size_t)q * a.hq + h;
+    load_row_bf16<D>(a.q + row * D, x);
     qk_prologue_bwd<D>(x, g, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps);
-    float4 *dst = reinterpret_cast<float4 *>(a.dq + (size_t)row * D);
+    float4 *dst = reinterpret_cast<float4 *>(a.dq + row * D);
 #pragma unroll
     for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(g[4 * c], g[4 * c + 1], g[4 * c + 2], g[4 * c + 3]);
 }
@@ -648,7 +714,9 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     auto *lse2 = reinterpret_cast<float *>(ws + 2 * kvb + 2 * qb);
     auto *dsum = reinterpret_cast<float *>(ws + 2 * kvb + 2 * qb + vb);
     auto *bounds = reinterpret_cast<float *>(ws + 2 * kvb + 2 * qb + 2 * vb);
+    auto *dqacc = reinterpret_cast<float *>(ws + 2 * kvb + 2 * qb + 2 * vb + 256);
     if (cudaMemsetAsync(bounds, 0, 2 * sizeof(float), stream) != cudaSuccess) return BCA_ERR_CUDA;
+    if (cudaMemsetAsync(dqacc, 0, dq_acc_bytes(P), stream) != cudaSuccess) return BCA_ERR_CUDA;
 
     PrepArgs pa;
     pa.q = static_cast<const __nv_bfloat16 *>(io.q);
@@ -672,7 +740,6 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     pa.bounds = bounds;
     pa.lse2 = lse2;
     pa.dsum = dsum;
-    pa.dq = io.dq;
     {
         ProfScope ps(P, BCA_KERNEL_BWD_PREP, stream);
         bwd_prep_kernel<D><<<dim3((unsigned)P.nqt, (unsigned)P.hq), 128, 0, stream>>>(pa);
@@ -731,7 +798,7 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     ba.hq = P.hq;
     ba.hkv = P.hkv;
     ba.eps = P.eps;
-    ba.dq = io.dq;
+    ba.dqacc = dqacc;
     ba.dk = io.dk;
     ba.dv = io.dv;
     ba.dkc = io.dk_cache;
@@ -754,15 +821,16 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     da.off1 = P.rope_axis_off[1];
     da.off2 = P.rope_axis_off[2];
     da.nq = P.nq;
+    da.nqt = P.nqt;
     da.hq = P.hq;
     da.eps = P.eps;
     da.scale = 1.0f / sqrtf((float)D);
     da.dq = io.dq;
+    da.dqacc = dqacc;
     da.bounds = bounds;
     {
         ProfScope ps(P, BCA_KERNEL_BWD_DQ, stream);
-        const int64_t rows = P.nq * P.hq;
-        bwd_dq_kernel<D><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(da);
+        if (P.nq > 0) bwd_dq_kernel<D><<<dim3((unsigned)P.nqt, (unsigned)P.hq), 128, 0, stream>>>(da);
     }
     if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
     (void)DPAD;
@@ -781,8 +849,10 @@ size_t q_vector_bytes(const Plan &P) {
     return (b + 255) / 256 * 256;
 }
 
+size_t dq_acc_bytes(const Plan &P) { return (size_t)P.hq * (size_t)P.nqt * 128 * (size_t)P.dpad * 4; }
+
 size_t bwd_workspace_bytes(const Plan &P) {
-    return 2 * kv_image_bytes(P) + 2 * q_image_bytes(P) + 2 * q_vector_bytes(P) + 256;
+    return 2 * kv_image_bytes(P) + 2 * q_image_bytes(P) + 2 * q_vector_bytes(P) + 256 + dq_acc_bytes(P);
 }
 
 int launch_bwd(Plan &P, const BwdIO &io, cudaStream_t stream) {

@@ -275,7 +275,8 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
             }
             // every issued copy must have landed before the CTA may exit
             for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
-                mbar_wait(bar(L::B_KV_FULL + j % STAGES), (j / STAGES) & 1, a.timeout_ns);
+                if (!mbar_wait(bar(L::B_KV_FULL + j % STAGES), (j / STAGES) & 1, a.timeout_ns))
+                    record_timeout(a.status, abort_flag);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -338,7 +339,7 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
             }
             // all issued MMAs must be complete before TMEM is released
             mma_commit(bar(L::B_MMA_DONE));
-            mbar_wait(bar(L::B_MMA_DONE), 0, a.timeout_ns);
+            if (!mbar_wait(bar(L::B_MMA_DONE), 0, a.timeout_ns)) record_timeout(a.status, abort_flag);
         }
         __syncwarp();
     } else if (warp >= 4) {

@@ -35,6 +35,8 @@ size_t fwd_workspace_bytes(const Plan &plan);
 // per-query vector (LSE, Dsum); and the whole backward workspace.
 size_t q_image_bytes(const Plan &plan);
 size_t q_vector_bytes(const Plan &plan);
+// Bytes of the backward's fp32 dQ-hat accumulator ([Hq][query tile][2][128][Dpad / 2]).
+size_t dq_acc_bytes(const Plan &plan);
 size_t bwd_workspace_bytes(const Plan &plan);
 
 // Bracket a launch with events when the plan is profiling (no-op otherwise).
