@@ -34,7 +34,9 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
+#include <type_traits>
 
 #include "kernels.hpp"
 #include "prologue.cuh"
@@ -117,13 +119,17 @@ struct DqArgs {
     float *dq;
 };
 
-// Power-of-two scale applied to dS before its fp16 rounding: 1 unless the bound
+// Power-of-two scale sc applied to dS before its fp16 rounding: 1 unless the bound
 // 2 max|dO| max|v| on |dS| exceeds 2^14, else the power of two bringing it below.
-__device__ __forceinline__ float ds_scale(const float *bounds) {
+// ds_scale_log2 gives log2(sc), an integer in [-100, 0]; ds_scale builds sc from its bits.
+__device__ __forceinline__ int ds_scale_log2(const float *bounds) {
     const float b = 2.0f * __ldg(bounds) * __ldg(bounds + 1);
-    if (!(b > 16384.0f)) return 1.0f;
+    if (!(b > 16384.0f)) return 0;
     const float e = ceilf(log2f(b * (1.0f / 16384.0f)) + 1e-3f);
-    return exp2f(-fminf(e, 100.0f));
+    return -(int)fminf(e, 100.0f);
+}
+__device__ __forceinline__ float ds_scale(const float *bounds) {
+    return __int_as_float((127 + ds_scale_log2(bounds)) << 23);
 }
 
 // atomic max of non-negative floats through their (order-preserving) bit patterns
@@ -202,8 +208,10 @@ __global__ void __launch_bounds__(128) bwd_prep_kernel(PrepArgs a) {
         const float L = a.lse[(size_t)h * a.nq + q];
         if (L > -INFINITY) lse2 = L * kLog2e;  // a row with no visible key keeps +inf: P = 0
     }
-    a.lse2[((size_t)h * a.nqt + qt) * 128 + t] = lse2;
-    a.dsum[((size_t)h * a.nqt + qt) * 128 + t] = dsum;
+    // stored negated, so the main kernel forms S - LSE and dP - Dsum with additions;
+    // bwd_shift_kernel later adds log2 of the dS scale to -LSE
+    a.lse2[((size_t)h * a.nqt + qt) * 128 + t] = -lse2;
+    a.dsum[((size_t)h * a.nqt + qt) * 128 + t] = -dsum;
 }
 
 template <int D>
@@ -246,6 +254,15 @@ __global__ void __launch_bounds__(128) bwd_kv_image_kernel(BwdKVArgs a) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if ((t & 31) == 0) atomic_max_nonneg(a.bounds + 1, m);
+}
+
+// -LSE2 += log2(sc): the main kernel then forms P sc = exp2(S - LSE2 + log2 sc) directly
+// (sc a power of two, so dV, accumulated from bf16(P sc), is undone exactly)
+__global__ void __launch_bounds__(256) bwd_shift_kernel(float *nlse2, int64_t count, const float *bounds) {
+    const int e = ds_scale_log2(bounds);  // 0 in the common case
+    if (e == 0) return;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x)
+        nlse2[i] += (float)e;
 }
 
 // ------------------------------------------------------------------ main kernel
@@ -544,8 +561,8 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
             tc_fence_before();
             mbar_arrive(bar(L::B_S_FREE));
 
-            const float4 *lse4 = reinterpret_cast<const float4 *>(st + L::ST_LSE) + c0 / 4;
-            const float4 *dsum4 = reinterpret_cast<const float4 *>(st + L::ST_DSUM) + c0 / 4;
+            const float4 *nlse4 = reinterpret_cast<const float4 *>(st + L::ST_LSE) + c0 / 4;
+            const float4 *ndsum4 = reinterpret_cast<const float4 *>(st + L::ST_DSUM) + c0 / 4;
             const bool partial = cur.r->mask_idx >= 0;
             const uint32_t *mask = reinterpret_cast<const uint32_t *>(st + L::ST_MASK);
             const int b = i & 1;
@@ -559,35 +576,50 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                 tc_fence_after();
             }
             uint4 *dsb = dsb0 + b * 2048;
-            // P = exp2(S - LSE) and dS = P (dP - Dsum), 16 columns at a time: P as bf16
-            // pairs into tensor memory, dS as fp16 into the dS^T image
+            // P sc = exp2(S - LSE + log2 sc) and dS sc = P sc (dP - Dsum), 16 columns at a
+            // time in paired fp32 arithmetic (the vectors come negated): P sc as bf16 pairs
+            // into tensor memory, dS sc as fp16 into the dS^T image.  The mask test is
+            // compiled into a separate copy for partial tiles.
+            auto emit = [&](auto partial_c) {
+                constexpr bool PARTIAL = decltype(partial_c)::value;
 #pragma unroll
-            for (int k2 = 0; k2 < 4; ++k2) {
-                uint32_t pw[8];
+                for (int k2 = 0; k2 < 4; ++k2) {
+                    uint32_t pw[8];
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const int k = 2 * k2 + hf;
-                    const float4 l0 = lse4[2 * k], l1 = lse4[2 * k + 1], d0 = dsum4[2 * k], d1 = dsum4[2 * k + 1];
-                    const float lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
-                    const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-                    uint32_t dw[4];
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const int k = 2 * k2 + hf;
+                        const float4 l0 = nlse4[2 * k], l1 = nlse4[2 * k + 1];
+                        const float4 d0 = ndsum4[2 * k], d1 = ndsum4[2 * k + 1];
+                        const float2 lv[4] = {make_float2(l0.x, l0.y), make_float2(l0.z, l0.w),
+                                              make_float2(l1.x, l1.y), make_float2(l1.z, l1.w)};
+                        const float2 dv[4] = {make_float2(d0.x, d0.y), make_float2(d0.z, d0.w),
+                                              make_float2(d1.x, d1.y), make_float2(d1.z, d1.w)};
+                        uint32_t dw[4];
 #pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        const int c = 8 * k + e;
-                        float p0 = ex2(__uint_as_float(su[c]) - lv[e]);
-                        float p1 = ex2(__uint_as_float(su[c + 1]) - lv[e + 1]);
-                        if (partial) {
-                            if (!((mask[(c0 + c) * 4 + r / 32] >> (r % 32)) & 1u)) p0 = 0.f;
-                            if (!((mask[(c0 + c + 1) * 4 + r / 32] >> (r % 32)) & 1u)) p1 = 0.f;
+                        for (int e = 0; e < 4; ++e) {
+                            const int c = 8 * k + 2 * e;
+                            const float2 x =
+                                __fadd2_rn(make_float2(__uint_as_float(su[c]), __uint_as_float(su[c + 1])), lv[e]);
+                            float2 p = make_float2(ex2(x.x), ex2(x.y));
+                            if constexpr (PARTIAL) {
+                                if (!((mask[(c0 + c) * 4 + r / 32] >> (r % 32)) & 1u)) p.x = 0.f;
+                                if (!((mask[(c0 + c + 1) * 4 + r / 32] >> (r % 32)) & 1u)) p.y = 0.f;
+                            }
+                            const float2 t =
+                                __fadd2_rn(make_float2(__uint_as_float(du[c]), __uint_as_float(du[c + 1])), dv[e]);
+                            const float2 ds = __fmul2_rn(p, t);
+                            pw[4 * hf + e] = pack_bf16x2(p.x, p.y);
+                            dw[e] = pack_f16x2(ds.x, ds.y);
                         }
-                        pw[4 * hf + e / 2] = pack_bf16x2(p0, p1);
-                        dw[e / 2] = pack_f16x2(p0 * (__uint_as_float(du[c]) - dv[e]) * sc,
-                                               p1 * (__uint_as_float(du[c + 1]) - dv[e + 1]) * sc);
+                        dsb[img_chunk(c0 / 8 + k, r)] = make_uint4(dw[0], dw[1], dw[2], dw[3]);
                     }
-                    dsb[img_chunk(c0 / 8 + k, r)] = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+                    tmem_st8(tbase + lane_off + L::COL_PT + c0 / 2 + 8 * k2, pw);
                 }
-                tmem_st8(tbase + lane_off + L::COL_PT + c0 / 2 + 8 * k2, pw);
-            }
+            };
+            if (partial)
+                emit(std::true_type{});
+            else
+                emit(std::false_type{});
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
@@ -622,13 +654,14 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
         const int64_t key = kt * 128 + r;
         if (key < a.nk) {
             if (wg == 0) {
+                const float inv_sc = 1.0f / sc;  // exact: sc is a power of two
                 float *dst = key < a.nc ? (a.dvc ? a.dvc + ((size_t)key * a.hkv + g) * D : nullptr)
                                         : a.dv + ((size_t)(key - a.nc) * a.hkv + g) * D;
                 if (dst) {
 #pragma unroll
                     for (int c = 0; c < D / 4; ++c)
-                        reinterpret_cast<float4 *>(dst)[c] =
-                            make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+                        reinterpret_cast<float4 *>(dst)[c] = make_float4(acc[4 * c] * inv_sc, acc[4 * c + 1] * inv_sc,
+                                                                         acc[4 * c + 2] * inv_sc, acc[4 * c + 3] * inv_sc);
                 }
             } else {
                 float gk[D];
@@ -768,6 +801,15 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     {
         ProfScope ps(P, BCA_KERNEL_BWD_KV_IMAGE, stream);
         bwd_kv_image_kernel<D><<<dim3((unsigned)P.nkt, (unsigned)P.hkv), 128, 0, stream>>>(ka);
+    }
+    if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
+
+    {
+        // -LSE2 += log2 sc once the two bounds are final (no work when sc = 1)
+        const int64_t count = (int64_t)P.hq * P.nqt * 128;
+        const unsigned blocks = (unsigned)std::min<int64_t>((count + 255) / 256, 4 * 148);
+        ProfScope ps(P, BCA_KERNEL_BWD_PREP, stream);
+        if (count > 0) bwd_shift_kernel<<<blocks, 256, 0, stream>>>(lse2, count, bounds);
     }
     if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
 

@@ -93,6 +93,26 @@ def test_bwd_with_gains_random_slices_and_empty_rows():
             _err("dk_cache", dkc, rkc); _err("dv_cache", dvc, rvc)
 
 
+@pytest.mark.parametrize("name", ["tiny", "b45_replica"])
+def test_bwd_large_upstream_gradient(name):
+    """dO scaled by 2^12 (exact in bf16) pushes the bound 2 max|dO| max|v| on |dS| past
+    fp16's safe range, so the kernel applies a power-of-two scale to dS (and to P, through
+    the shifted LSE) and undoes it on dQ, dK, dV.  Gradients are linear in dO, so they
+    must equal 2^12 times the oracle's for the unscaled dO."""
+    w = W.WORKLOADS[name]
+    x = W.make_inputs(w, "cuda", with_grad=True)
+    x["do"] = x["do"] * 4096.0
+    dq, dk, dv, dkc, dvc = _gpu_fwd_bwd(w, x)
+    c = {k: (None if t is None else t.cpu()) for k, t in x.items()}
+    c["do"] = c["do"] / 4096.0
+    rq, rk, rv, rkc, rvc, _, _ = oracle.backward(c["q"], c["k"], c["v"], c["k_cache"], c["v_cache"], c["do"],
+                                                 w.videos_array(), w.slices_array(), w.hq, w.hkv,
+                                                 base=w.rope_base, eps=w.eps)
+    _err("dq", dq / 4096.0, rq); _err("dk", dk / 4096.0, rk); _err("dv", dv / 4096.0, rv)
+    if w.num_cache_keys:
+        _err("dk_cache", dkc / 4096.0, rkc); _err("dv_cache", dvc / 4096.0, rvc)
+
+
 @pytest.mark.parametrize("name,nrows", [("p720_pipelined", 24), ("packed_varlen", 24), ("long_kvrange", 12)])
 def test_bwd_full_size_sampled_dq_and_dv_sums(name, nrows):
     """Full-size workloads in the benchmark's launch configuration: dq on a seeded row
