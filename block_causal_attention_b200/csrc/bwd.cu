@@ -552,14 +552,13 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                  warp_wait_abort(bar(L::B_S_FULL), i & 1, a.status, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            uint32_t su[64], du[64];  // S^T and dP^T values of this thread's 64 columns (raw bits)
-            tmem_ld32(tbase + lane_off + L::COL_S + c0, *reinterpret_cast<uint32_t(*)[32]>(&su[0]));
-            tmem_ld32(tbase + lane_off + L::COL_S + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&su[32]));
-            tmem_ld32(tbase + lane_off + L::COL_DP + c0, *reinterpret_cast<uint32_t(*)[32]>(&du[0]));
-            tmem_ld32(tbase + lane_off + L::COL_DP + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&du[32]));
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(bar(L::B_S_FREE));
+            // S^T / dP^T leave tensor memory 16 columns at a time, the next chunk in flight
+            // while the current one is processed (two register buffers)
+            const uint32_t tS = tbase + lane_off + L::COL_S + c0, tDP = tbase + lane_off + L::COL_DP + c0;
+            const uint32_t tPT = tbase + lane_off + L::COL_PT + c0 / 2;
+            uint32_t sv[2][16], pv[2][16];
+            tmem_ld16(tS, sv[0]);
+            tmem_ld16(tDP, pv[0]);
 
             const float4 *nlse4 = reinterpret_cast<const float4 *>(st + L::ST_LSE) + c0 / 4;
             const float4 *ndsum4 = reinterpret_cast<const float4 *>(st + L::ST_DSUM) + c0 / 4;
@@ -568,26 +567,34 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
             const int b = i & 1;
             if (i > 1) {  // dS^T buffer b was last read by the dK / dQ MMAs of item i - 2
                 ok = warp_wait_abort(bar(L::B_DS_FREE + b), ((i >> 1) - 1) & 1, a.status, abort_flag);
-                if (!ok) break;
             }
-            if (i > 0) {  // the dV MMAs of item i - 1 have read P^T from tensor memory
+            if (ok && i > 0) {  // the dV MMAs of item i - 1 have read P^T from tensor memory
                 ok = warp_wait_abort(bar(L::B_PT_FREE), (i - 1) & 1, a.status, abort_flag);
-                if (!ok) break;
                 tc_fence_after();
             }
+            if (!ok) {
+                tmem_wait_ld();
+                break;
+            }
             uint4 *dsb = dsb0 + b * 2048;
-            // P sc = exp2(S - LSE + log2 sc) and dS sc = P sc (dP - Dsum), 16 columns at a
-            // time in paired fp32 arithmetic (the vectors come negated): P sc as bf16 pairs
-            // into tensor memory, dS sc as fp16 into the dS^T image.  The mask test is
-            // compiled into a separate copy for partial tiles.
+            // P sc = exp2(S - LSE + log2 sc) and dS sc = P sc (dP - Dsum) in paired fp32
+            // arithmetic (the vectors come negated): P sc as bf16 pairs into tensor memory,
+            // dS sc as fp16 into the dS^T image.  The mask test is compiled into a separate
+            // copy for partial tiles.
             auto emit = [&](auto partial_c) {
                 constexpr bool PARTIAL = decltype(partial_c)::value;
+                tmem_wait_ld_regs(sv[0], pv[0]);
 #pragma unroll
-                for (int k2 = 0; k2 < 4; ++k2) {
+                for (int q = 0; q < 4; ++q) {
+                    const int cb = q & 1;
+                    if (q < 3) {
+                        tmem_ld16(tS + 16 * (q + 1), sv[cb ^ 1]);
+                        tmem_ld16(tDP + 16 * (q + 1), pv[cb ^ 1]);
+                    }
                     uint32_t pw[8];
 #pragma unroll
                     for (int hf = 0; hf < 2; ++hf) {
-                        const int k = 2 * k2 + hf;
+                        const int k = 2 * q + hf;
                         const float4 l0 = nlse4[2 * k], l1 = nlse4[2 * k + 1];
                         const float4 d0 = ndsum4[2 * k], d1 = ndsum4[2 * k + 1];
                         const float2 lv[4] = {make_float2(l0.x, l0.y), make_float2(l0.z, l0.w),
@@ -597,23 +604,29 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                         uint32_t dw[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const int c = 8 * k + 2 * e;
-                            const float2 x =
-                                __fadd2_rn(make_float2(__uint_as_float(su[c]), __uint_as_float(su[c + 1])), lv[e]);
+                            const int c = 8 * hf + 2 * e;  // column within the chunk
+                            const float2 x = __fadd2_rn(
+                                make_float2(__uint_as_float(sv[cb][c]), __uint_as_float(sv[cb][c + 1])), lv[e]);
                             float2 p = make_float2(ex2(x.x), ex2(x.y));
                             if constexpr (PARTIAL) {
-                                if (!((mask[(c0 + c) * 4 + r / 32] >> (r % 32)) & 1u)) p.x = 0.f;
-                                if (!((mask[(c0 + c + 1) * 4 + r / 32] >> (r % 32)) & 1u)) p.y = 0.f;
+                                const int col = c0 + 16 * q + c;
+                                if (!((mask[col * 4 + r / 32] >> (r % 32)) & 1u)) p.x = 0.f;
+                                if (!((mask[(col + 1) * 4 + r / 32] >> (r % 32)) & 1u)) p.y = 0.f;
                             }
-                            const float2 t =
-                                __fadd2_rn(make_float2(__uint_as_float(du[c]), __uint_as_float(du[c + 1])), dv[e]);
+                            const float2 t = __fadd2_rn(
+                                make_float2(__uint_as_float(pv[cb][c]), __uint_as_float(pv[cb][c + 1])), dv[e]);
                             const float2 ds = __fmul2_rn(p, t);
                             pw[4 * hf + e] = pack_bf16x2(p.x, p.y);
                             dw[e] = pack_f16x2(ds.x, ds.y);
                         }
                         dsb[img_chunk(c0 / 8 + k, r)] = make_uint4(dw[0], dw[1], dw[2], dw[3]);
                     }
-                    tmem_st8(tbase + lane_off + L::COL_PT + c0 / 2 + 8 * k2, pw);
+                    tmem_st8(tPT + 8 * q, pw);
+                    if (q < 3) tmem_wait_ld_regs(sv[cb ^ 1], pv[cb ^ 1]);
+                    if (q == 2) {  // every S^T / dP^T value of this thread is in registers
+                        tc_fence_before();
+                        mbar_arrive(bar(L::B_S_FREE));
+                    }
                 }
             };
             if (partial)
