@@ -356,10 +356,13 @@ def run_ours(a):
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    tpath = os.path.join(ROOT, "profiles", "traffic.txt")
     if os.path.exists(tpath):
         with open(tpath) as f:
-            traffic = json.load(f).get(f"{dom}:{w.name}")
+            for line in f:
+                parts = line.split()
+                if len(parts) >= 3 and not parts[0].startswith("#") and parts[0] == dom and parts[1] == w.name:
+                    traffic = float(parts[2])
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
                 "frac": achieved / peak_sus, "traffic": traffic,
                 "kernel": dom, "peak_kind": f"bf16 dense, sustained, {peak_src}",
