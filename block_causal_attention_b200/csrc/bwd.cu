@@ -427,20 +427,53 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t k16 = sbase + L::OFF_K16, vb = sbase + L::OFF_V;
-            const uint32_t dst0 = sbase + L::OFF_DST;
-            auto stage = [&](int i) -> uint32_t { return sbase + L::OFF_STAGE + (i % STAGES) * L::STAGE_BYTES; };
+            // descriptors built once, advanced by constants (the address field is the low 14
+            // bits of the byte address / 16, so adding offset / 16 is exact)
+            const uint64_t dk16 = smem_desc(sbase + L::OFF_K16, 2048, 128);      // K-hat, K-major A of S^T
+            const uint64_t dvk = smem_desc(sbase + L::OFF_V, 2048, 128);         // V, K-major A of dP^T
+            const uint64_t dkmn = smem_desc(sbase + L::OFF_K16, 128, 2048);      // K-hat, MN-major B of dQ
+            const uint64_t dq_k = smem_desc(sbase + L::OFF_STAGE + L::ST_Q16, 2048, 128);  // Q-hat, K-major B of S^T
+            const uint64_t ddo_k = smem_desc(sbase + L::OFF_STAGE + L::ST_DO, 2048, 128);  // dO, K-major B of dP^T
+            const uint64_t dq_mn = smem_desc(sbase + L::OFF_STAGE + L::ST_Q16, 128, 2048); // Q-hat, MN-major B of dK
+            const uint64_t ddo_mn = smem_desc(sbase + L::OFF_STAGE + L::ST_DO, 128, 2048); // dO, MN-major B of dV
+            const uint64_t dds_k = smem_desc(sbase + L::OFF_DST, 2048, 128);     // dS^T, K-major A of dK
+            const uint64_t dds_mn = smem_desc(sbase + L::OFF_DST, 128, 2048);    // dS^T, MN-major A of dQ
+            auto stoff = [&](int i) -> uint64_t { return (uint64_t)(((i % STAGES) * L::STAGE_BYTES) >> 4); };
             // S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 128 queries, K = DPAD; all K-major)
             auto issue_s_dp = [&](int i) {
-                const uint32_t st = stage(i);
+                const uint64_t so = stoff(i);
 #pragma unroll
                 for (int kk = 0; kk < DPAD / 16; ++kk)
-                    mma_f16(tbase + L::COL_S, smem_desc(k16 + kk * 4096, 2048, 128),
-                            smem_desc(st + L::ST_Q16 + kk * 4096, 2048, 128), IDESC_S, kk > 0);
+                    mma_f16(tbase + L::COL_S, dk16 + (uint64_t)(kk * 256), dq_k + so + (uint64_t)(kk * 256), IDESC_S,
+                            kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < DPAD / 16; ++kk)
-                    mma_f16(tbase + L::COL_DP, smem_desc(vb + kk * 4096, 2048, 128),
-                            smem_desc(st + L::ST_DO + kk * 4096, 2048, 128), IDESC_DP, kk > 0);
+                    mma_f16(tbase + L::COL_DP, dvk + (uint64_t)(kk * 256), ddo_k + so + (uint64_t)(kk * 256), IDESC_DP,
+                            kk > 0);
+            };
+            // dV += P^T dO (A = P^T in tensor memory, B MN-major dO) and dK += dS^T Q (A K-major
+            // dS^T, B MN-major Q-hat)
+            auto issue_dv = [&](int i) {
+                const uint64_t so = stoff(i);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16_ts(tbase + L::COL_DV, tbase + L::COL_PT + 8 * kk, ddo_mn + so + (uint64_t)(kk * 16),
+                               IDESC_DV, (i > 0 || kk > 0) ? 1u : 0u);
+            };
+            auto issue_dk = [&](int i) {
+                const uint64_t so = stoff(i), bo = (uint64_t)(((i & 1) * 32768) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16(tbase + L::COL_DK, dds_k + bo + (uint64_t)(kk * 256), dq_mn + so + (uint64_t)(kk * 16),
+                            IDESC_DK, (i > 0 || kk > 0) ? 1u : 0u);
+            };
+            // dQ_part = dS K (A MN-major dS^T, B MN-major K-hat)
+            auto issue_dq = [&](int i) {
+                const uint64_t bo = (uint64_t)(((i & 1) * 32768) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16(tbase + L::COL_DQ, dds_mn + bo + (uint64_t)(kk * 16), dkmn + (uint64_t)(kk * 16), IDESC_DQ,
+                            kk > 0);
             };
             bool ok = wait_abort(bar(L::B_KV), 0, a.status, abort_flag);
             if (ok && n > 0) ok = wait_abort(bar(L::B_ST_FULL), 0, a.status, abort_flag);
@@ -450,7 +483,6 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                 mma_commit(bar(L::B_S_FULL));
             }
             for (int i = 0; i < n && ok; ++i) {
-                const uint32_t st = stage(i);
                 if (i + 1 < n) {
                     ok = wait_abort(bar(L::B_ST_FULL + (i + 1) % STAGES), ((i + 1) / STAGES) & 1, a.status,
                                     abort_flag) &&
@@ -461,34 +493,19 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                     mma_commit(bar(L::B_S_FULL));
                 }
                 const int b = i & 1;
-                const uint32_t dst = dst0 + b * 32768;
                 ok = wait_abort(bar(L::B_DS_READY), i & 1, a.status, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                // dV += P^T dO (M = 128 keys, N = DPAD, K = 128 queries): A = P^T in tensor
-                // memory (16 queries per 8 columns), B MN-major from the dO image
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_f16_ts(tbase + L::COL_DV, tbase + L::COL_PT + 8 * kk,
-                               smem_desc(st + L::ST_DO + kk * 256, 128, 2048), IDESC_DV, (i > 0 || kk > 0) ? 1u : 0u);
+                issue_dv(i);
                 mma_commit(bar(L::B_PT_FREE));
-                // dK += dS^T Q: A K-major from the dS^T buffer, B MN-major from the Q image
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_f16(tbase + L::COL_DK, smem_desc(dst + kk * 4096, 2048, 128),
-                            smem_desc(st + L::ST_Q16 + kk * 256, 128, 2048), IDESC_DK, (i > 0 || kk > 0) ? 1u : 0u);
+                issue_dk(i);
                 mma_commit(bar(L::B_ST_EMPTY + i % STAGES));
                 if (i > 0) {  // the compute warps have read dQ_part of item i - 1
                     ok = wait_abort(bar(L::B_DQ_FREE), (i - 1) & 1, a.status, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                 }
-                // dQ_part = dS K (M = 128 queries, N = DPAD, K = 128 keys): A MN-major from
-                // the dS^T buffer, B MN-major from the K image
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_f16(tbase + L::COL_DQ, smem_desc(dst + kk * 256, 128, 2048),
-                            smem_desc(k16 + kk * 256, 128, 2048), IDESC_DQ, kk > 0);
+                issue_dq(i);
                 mma_commit(bar(L::B_DQ_FULL));
                 mma_commit(bar(L::B_DS_FREE + b));
             }
