@@ -55,6 +55,8 @@ def lib():
         L.orc_prologue.argtypes = [_f64p, _i64, _int, _int, _i32p, _vp, _f64p, ctypes.c_double, _f64p]
         L.orc_prologue_bwd.argtypes = [_f64p, _i64, _int, _int, _i32p, _vp, _f64p, ctypes.c_double,
                                        _f64p, _f64p]
+        L.orc_prologue_param_grads.argtypes = [_f64p, _i64, _int, _int, _i32p, _vp, _f64p, ctypes.c_double,
+                                               _f64p, _f64p, _f64p]
         L.orc_fwd_rows.argtypes = [_f64p, _i64p, _i64, _f64p, _f64p, _i64, _i64p, _int, _int, _int,
                                    _int, _f64p, _f64p]
         L.orc_bwd_rows.argtypes = [_f64p, _i64p, _i64, _f64p, _f64p, _i64, _f64p, _i64p, _int, _int,
@@ -64,7 +66,7 @@ def lib():
         L.orc_bwd_dense.argtypes = [_f64p, _f64p, _f64p, _f64p, _i64, _i64, _i64p, _int, _int, _int,
                                     _int, _f64p, _f64p, _f64p, _f64p, _f64p]
         for f in ("orc_mask_row", "orc_mask_col", "orc_mask_dense", "orc_positions", "orc_prologue",
-                  "orc_prologue_bwd", "orc_fwd_rows", "orc_bwd_rows", "orc_bwd_keys", "orc_bwd_dense"):
+                  "orc_prologue_bwd", "orc_prologue_param_grads", "orc_fwd_rows", "orc_bwd_rows", "orc_bwd_keys", "orc_bwd_dense"):
             getattr(L, f).restype = None
         _lib = L
     return _lib
@@ -144,6 +146,21 @@ def prologue_bwd(x, pos, dy, base=(1e4, 1e4, 1e4), eps=1e-6, gain=None) -> np.nd
     lib().orc_prologue_bwd(x, n, H, D, pos, None if g is None else g.ctypes.data,
                            np.asarray(base, np.float64), float(eps), dy, out)
     return out
+
+
+def prologue_param_grads(x, pos, dy, base=(1e4, 1e4, 1e4), eps=1e-6, gain=None):
+    """(dL/dgain [D], dL/dbase [3]) of the prologue, summed over all rows of x [n, H, D]
+    for the upstream gradient dy = dL/d(prologue output)."""
+    x = _f64(x)
+    dy = _f64(dy)
+    n, H, D = x.shape
+    pos = np.ascontiguousarray(np.asarray(pos, dtype=np.int32).reshape(n, 3))
+    g = None if gain is None else _f64(gain)
+    dg = np.zeros(D)
+    db = np.zeros(3)
+    lib().orc_prologue_param_grads(x, n, H, D, pos, None if g is None else g.ctypes.data,
+                                   np.asarray(base, np.float64), float(eps), dy, dg, db)
+    return dg, db
 
 
 # ---------------------------------------------------------------------------
@@ -251,8 +268,10 @@ def forward(q, k, v, k_cache, v_cache, videos, slices, hq, hkv,
 
 
 def backward(q, k, v, k_cache, v_cache, do, videos, slices, hq, hkv,
-             base=(1e4, 1e4, 1e4), eps=1e-6, q_gain=None, k_gain=None):
-    """Full backward w.r.t. the raw inputs: (dq, dk, dv, dk_cache, dv_cache, O, LSE)."""
+             base=(1e4, 1e4, 1e4), eps=1e-6, q_gain=None, k_gain=None, param_grads=False):
+    """Full backward w.r.t. the raw inputs: (dq, dk, dv, dk_cache, dv_cache, O, LSE), and
+    with param_grads=True also (dq_gain [D], dk_gain [D], dbase [3]) appended: the
+    gradients of the two QK-Norm gains and of the RoPE bases (shared by Q and K)."""
     pos = positions(videos)
     nc = 0 if k_cache is None else int(k_cache.shape[0])
     kh = full_keys(prologue(k, pos, base, eps, k_gain), k_cache)
@@ -261,7 +280,12 @@ def backward(q, k, v, k_cache, v_cache, do, videos, slices, hq, hkv,
     dqh, dkh, dvv, O, lse = attn_bwd_dense(qh, kh, vv, do, slices, hq, hkv)
     dq = prologue_bwd(q, pos, dqh, base, eps, q_gain)
     dk = prologue_bwd(k, pos, dkh[nc:], base, eps, k_gain)
-    return dq, dk, dvv[nc:], (dkh[:nc] if nc else None), (dvv[:nc] if nc else None), O, lse
+    out = (dq, dk, dvv[nc:], (dkh[:nc] if nc else None), (dvv[:nc] if nc else None), O, lse)
+    if not param_grads:
+        return out
+    dgq, dbq = prologue_param_grads(q, pos, dqh, base, eps, q_gain)
+    dgk, dbk = prologue_param_grads(k, pos, dkh[nc:], base, eps, k_gain)
+    return out + (dgq, dgk, dbq + dbk)
 
 
 def backward_rows(q_rows, rows, k, v, k_cache, v_cache, do_rows, videos, slices, hq, hkv,

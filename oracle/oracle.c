@@ -185,6 +185,51 @@ void orc_prologue_bwd(const double *x, int64_t n, int H, int D, const int32_t *p
     }
 }
 
+/* Gradients of the prologue's parameters, accumulated (+=) over rows: the QK-Norm gain
+ * and the three RoPE bases (MAGI-1 research notes, "Autoregressive denoising DiT":
+ * QK-Norm, and 3D RoPE with a learnable base frequency).  dy = dL/d(out) per row.
+ * With z = x / r, xh = gain * z and y = R(angles) xh:
+ *   dL/dgain_d = sum over rows of (R^T dy)_d z_d;
+ *   for pair k of axis a, angle = pos_a * base_a^(-k/p), dy/dangle = (-y1, y0), so
+ *   dL/dangle = dy1 y0 - dy0 y1 and dangle/dbase_a = -(k/p) angle / base_a. */
+void orc_prologue_param_grads(const double *x, int64_t n, int H, int D, const int32_t *pos,
+                              const double *gain, const double *base, double eps,
+                              const double *dy, double *dgain, double *dbase)
+{
+    int p = (D / 2) / 3;
+    for (int64_t t = 0; t < n; ++t) {
+        for (int h = 0; h < H; ++h) {
+            const double *xr = x + ((size_t)t * H + h) * D;
+            const double *g = dy + ((size_t)t * H + h) * D;
+            double z[256], xh[256], dz[256];
+            double ss = 0.0;
+            for (int d = 0; d < D; ++d)
+                ss += xr[d] * xr[d];
+            double r = sqrt(ss / D + eps);
+            for (int d = 0; d < D; ++d) {
+                z[d] = xr[d] / r;
+                xh[d] = (gain ? gain[d] : 1.0) * z[d];
+                dz[d] = g[d];
+            }
+            for (int a = 0; a < 3; ++a) {
+                for (int k = 0; k < p; ++k) {
+                    int c0 = 2 * p * a + 2 * k;
+                    double ang = rope_angle(pos[3 * t + a], base[a], k, p);
+                    double cs = cos(ang), sn = sin(ang);
+                    double y0 = xh[c0] * cs - xh[c0 + 1] * sn;
+                    double y1 = xh[c0] * sn + xh[c0 + 1] * cs;
+                    double dang = g[c0 + 1] * y0 - g[c0] * y1;
+                    dbase[a] += dang * (-(double)k / (double)p) * ang / base[a];
+                    dz[c0] = g[c0] * cs + g[c0 + 1] * sn;
+                    dz[c0 + 1] = -g[c0] * sn + g[c0 + 1] * cs;
+                }
+            }
+            for (int d = 0; d < D; ++d)
+                dgain[d] += dz[d] * z[d];
+        }
+    }
+}
+
 /* One (row, head): scores over the visible keys, LSE and O.  Returns LSE (-inf when
  * the row sees no key, with O = 0). */
 static double attend_row(const double *q, const double *kh, const double *v, int64_t nk,

@@ -331,6 +331,39 @@ def test_backward_matches_central_finite_differences():
             assert abs(fd - g[ix]) <= 1e-6 * max(1.0, abs(fd)), (ai, ix, fd, g[ix])
 
 
+@pytest.mark.parametrize("D", [24, 32])
+def test_parameter_gradients_match_central_finite_differences(D):
+    """Gradients of the QK-Norm gains (Q and K) and of the three RoPE bases against
+    central differences of the forward in fp64.  D = 32 leaves one pair unrotated, and
+    the cache keys (already post-prologue) must not contribute to the K gain."""
+    Hq, Hkv = 4, 2
+    videos = np.asarray([[2, 1, 2, 3, 4]], np.int32)
+    nq, nc = 12, 6
+    sl = _block_causal([2], 6, cache=nc)
+    q, k, v = _rand((nq, Hq, D)), _rand((nq, Hkv, D)), _rand((nq, Hkv, D))
+    kc, vc = _rand((nc, Hkv, D)), _rand((nc, Hkv, D))
+    R = _rand((nq, Hq, D))
+    g_q, g_k = RNG.uniform(0.5, 1.5, D), RNG.uniform(0.5, 1.5, D)
+    base = np.asarray([100.0, 50.0, 20.0])
+
+    def loss(gq, gk, b):
+        O, _ = oracle.forward(q, k, v, kc, vc, videos, sl, Hq, Hkv, base=tuple(b), q_gain=gq, k_gain=gk)
+        return float((O * R).sum())
+
+    out = oracle.backward(q, k, v, kc, vc, R, videos, sl, Hq, Hkv, base=tuple(base), q_gain=g_q,
+                          k_gain=g_k, param_grads=True)
+    dgq, dgk, db = out[7], out[8], out[9]
+    for name, vec, grad in (("q_gain", 0, dgq), ("k_gain", 1, dgk), ("base", 2, db)):
+        for i in range(len(grad)):
+            vals = [g_q.copy(), g_k.copy(), base.copy()]
+            h = 1e-6 * max(1.0, abs(vals[vec][i]))
+            vp = [x.copy() for x in vals]; vp[vec][i] += h
+            vm = [x.copy() for x in vals]; vm[vec][i] -= h
+            fd = (loss(*vp) - loss(*vm)) / (2 * h)
+            assert abs(fd - grad[i]) <= 2e-6 * max(1.0, abs(fd)), (name, i, fd, grad[i])
+    assert np.any(np.abs(db) > 1e-3) and np.any(np.abs(dgk) > 1e-3)
+
+
 def test_backward_dv_sums_to_do_sum():
     """Rows of P sum to one, so sum_j dV_j = sum over the group's heads and rows with a
     visible key of dO_i; and sum_j dS_ij = 0, so sum_j dkh_j = 0 per group."""
