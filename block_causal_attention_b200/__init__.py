@@ -117,9 +117,12 @@ class Plan:
         return o, lse
 
     def bwd(self, q, k, v, k_cache, v_cache, o, lse, dout, *, dq=None, dk=None, dv=None, dk_cache=None,
-            dv_cache=None, workspace=None, q_gain=None, k_gain=None, stream=None, want_cache_grads=True):
+            dv_cache=None, workspace=None, q_gain=None, k_gain=None, stream=None, want_cache_grads=True,
+            param_grads=False):
         """Gradients (fp32) w.r.t. q, k, v (new tokens, through QK-Norm + RoPE) and the
-        cache; o, lse are the forward's outputs, dout the upstream gradient of O."""
+        cache; o, lse are the forward's outputs, dout the upstream gradient of O.
+        Returns (dq, dk, dv, dk_cache, dv_cache), and with param_grads=True also
+        (dq_gain [D], dk_gain [D], drope_base [3]) appended."""
         import torch
         if self.host_only:
             raise BcaError(_abi.BCA_ERR_HOST_ONLY_PLAN, "bwd")
@@ -137,11 +140,21 @@ class Plan:
             dv_cache = torch.empty(shp, device=dev, dtype=f32) if dv_cache is None else dv_cache
         if workspace is None:
             workspace = self.alloc_workspace(_abi.BCA_PASS_BWD)
-        rc = self._lib.bca_bwd(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(q_gain),
-                               _ptr(k_gain), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
-                               _ptr(dk_cache), _ptr(dv_cache), _ptr(workspace), self._stream(stream))
-        _abi.check(rc, "bca_bwd")
-        return dq, dk, dv, dk_cache, dv_cache
+        if not param_grads:
+            rc = self._lib.bca_bwd(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(q_gain),
+                                   _ptr(k_gain), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                   _ptr(dk_cache), _ptr(dv_cache), _ptr(workspace), self._stream(stream))
+            _abi.check(rc, "bca_bwd")
+            return dq, dk, dv, dk_cache, dv_cache
+        dgq = torch.empty(self.d, device=dev, dtype=f32)
+        dgk = torch.empty(self.d, device=dev, dtype=f32)
+        dbase = torch.empty(3, device=dev, dtype=f32)
+        rc = self._lib.bca_bwd_ex(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(q_gain),
+                                  _ptr(k_gain), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                  _ptr(dk_cache), _ptr(dv_cache), _ptr(dgq), _ptr(dgk), _ptr(dbase),
+                                  _ptr(workspace), self._stream(stream))
+        _abi.check(rc, "bca_bwd_ex")
+        return dq, dk, dv, dk_cache, dv_cache, dgq, dgk, dbase
 
     def profile(self, enable: bool = True) -> None:
         """Bracket every kernel launched for this plan with CUDA events."""

@@ -36,6 +36,7 @@ ProfScope::~ProfScope() {
 namespace {
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -193,10 +194,10 @@ int bca_fwd(bca_plan_t plan, const void *q, const void *k, const void *v, const 
     return bca::launch_fwd(P, io, static_cast<cudaStream_t>(stream));
 }
 
-int bca_bwd(bca_plan_t plan, const void *q, const void *k, const void *v, const void *k_cache,
-            const void *v_cache, const float *q_gain, const float *k_gain, const void *o, const float *lse,
-            const void *dout, float *dq, float *dk, float *dv, float *dk_cache, float *dv_cache,
-            void *workspace, void *stream) {
+int bca_bwd_ex(bca_plan_t plan, const void *q, const void *k, const void *v, const void *k_cache,
+               const void *v_cache, const float *q_gain, const float *k_gain, const void *o, const float *lse,
+               const void *dout, float *dq, float *dk, float *dv, float *dk_cache, float *dv_cache,
+               float *dq_gain, float *dk_gain, float *drope_base, void *workspace, void *stream) {
     if (!plan) return BCA_ERR_INVALID_ARGUMENT;
     bca::Plan &P = plan->plan;
     int rc = check_device(P);
@@ -207,6 +208,9 @@ int bca_bwd(bca_plan_t plan, const void *q, const void *k, const void *v, const 
         const size_t cb = (size_t)P.nc * P.hkv * P.d * sizeof(float);
         if (dk_cache && cudaMemsetAsync(dk_cache, 0, cb, s) != cudaSuccess) return BCA_ERR_CUDA;
         if (dv_cache && cudaMemsetAsync(dv_cache, 0, cb, s) != cudaSuccess) return BCA_ERR_CUDA;
+        if (dq_gain && cudaMemsetAsync(dq_gain, 0, P.d * sizeof(float), s) != cudaSuccess) return BCA_ERR_CUDA;
+        if (dk_gain && cudaMemsetAsync(dk_gain, 0, P.d * sizeof(float), s) != cudaSuccess) return BCA_ERR_CUDA;
+        if (drope_base && cudaMemsetAsync(drope_base, 0, 3 * sizeof(float), s) != cudaSuccess) return BCA_ERR_CUDA;
         return BCA_OK;
     }
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return BCA_ERR_INVALID_ARGUMENT;
@@ -215,8 +219,20 @@ int bca_bwd(bca_plan_t plan, const void *q, const void *k, const void *v, const 
                           workspace};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return BCA_ERR_MISALIGNED;
-    bca::BwdIO io{q, k, v, k_cache, v_cache, q_gain, k_gain, o, lse, dout, dq, dk, dv, dk_cache, dv_cache, workspace};
+    const void *pptrs[] = {dq_gain, dk_gain, drope_base};
+    for (const void *p : pptrs)
+        if (p && !aligned4(p)) return BCA_ERR_MISALIGNED;
+    bca::BwdIO io{q,  k,  v,  k_cache,  v_cache,  q_gain,    k_gain,  o,       lse,       dout,      dq,
+                  dk, dv, dk_cache, dv_cache, workspace, dq_gain, dk_gain, drope_base};
     return bca::launch_bwd(P, io, s);
+}
+
+int bca_bwd(bca_plan_t plan, const void *q, const void *k, const void *v, const void *k_cache,
+            const void *v_cache, const float *q_gain, const float *k_gain, const void *o, const float *lse,
+            const void *dout, float *dq, float *dk, float *dv, float *dk_cache, float *dv_cache,
+            void *workspace, void *stream) {
+    return bca_bwd_ex(plan, q, k, v, k_cache, v_cache, q_gain, k_gain, o, lse, dout, dq, dk, dv, dk_cache, dv_cache,
+                      nullptr, nullptr, nullptr, workspace, stream);
 }
 
 int bca_profile_enable(bca_plan_t plan, int enable) {

@@ -102,6 +102,8 @@ struct BwdArgs {
     float eps;
     float *dqacc;  // fp32 dQ-hat accumulator, [Hq][query tile][2][128][DPAD / 2]
     float *dk, *dv, *dkc, *dvc;
+    float *dgain_k, *dbase;  // optional parameter gradients (K gain; RoPE bases, shared with Q)
+    float coef[24];          // d(base_a^(-k/P))/d(base_a) at [8 a + k]
     int *status;
 };
 
@@ -117,6 +119,8 @@ struct DqArgs {
     const float *bounds;
     const float *dqacc;
     float *dq;
+    float *dgain_q, *dbase;  // optional parameter gradients (Q gain; RoPE bases, shared with K)
+    float coef[24];
 };
 
 // Power-of-two scale sc applied to dS before its fp16 rounding: 1 unless the bound
@@ -263,6 +267,28 @@ __global__ void __launch_bounds__(256) bwd_shift_kernel(float *nlse2, int64_t co
     if (e == 0) return;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x)
         nlse2[i] += (float)e;
+}
+
+// Sum the D + 3 parameter-gradient partials of a warp's 32 rows and add them to
+// dgain [D] and dbase [3] (lane 0; a NULL target is skipped).
+template <int D>
+__device__ __forceinline__ void warp_param_grads_add(float (&pg)[D], float (&pb)[3], float *dgain, float *dbase) {
+#pragma unroll
+    for (int d = 0; d < D; ++d)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) pg[d] += __shfl_xor_sync(0xffffffffu, pg[d], o);
+#pragma unroll
+    for (int e = 0; e < 3; ++e)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) pb[e] += __shfl_xor_sync(0xffffffffu, pb[e], o);
+    if ((threadIdx.x & 31) == 0) {
+        if (dgain)
+#pragma unroll
+            for (int d = 0; d < D; ++d) atomicAdd(dgain + d, pg[d]);
+        if (dbase)
+#pragma unroll
+            for (int e = 0; e < 3; ++e) atomicAdd(dbase + e, pb[e]);
+    }
 }
 
 // ------------------------------------------------------------------ main kernel
@@ -682,6 +708,10 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
             }
         }
         const int64_t key = kt * 128 + r;
+        const bool want_pg = wg == 1 && (a.dgain_k != nullptr || a.dbase != nullptr);
+        float pg[D], pb[3] = {0.f, 0.f, 0.f};  // parameter-gradient partials of this key row
+#pragma unroll
+        for (int d = 0; d < D; ++d) pg[d] = 0.f;
         if (key < a.nk) {
             if (wg == 0) {
                 const float inv_sc = 1.0f / sc;  // exact: sc is a power of two
@@ -704,6 +734,9 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                     const int64_t nn = key - a.nc;
                     float x[D];
                     load_row_bf16<D>(a.k + ((size_t)nn * a.hkv + g) * D, x);
+                    if (want_pg)
+                        qk_param_grads<D>(x, gk, __ldg(a.pos + nn), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps,
+                                          a.coef, pg, pb);
                     qk_prologue_bwd<D>(x, gk, __ldg(a.pos + nn), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps);
                     dst = a.dk + ((size_t)nn * a.hkv + g) * D;
                 }
@@ -714,6 +747,7 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                 }
             }
         }
+        if (want_pg) warp_param_grads_add<D>(pg, pb, a.dgain_k, a.dbase);
     }
 
     tc_fence_before();
@@ -732,34 +766,72 @@ __global__ void __launch_bounds__(128) bwd_dq_kernel(DqArgs a) {
     constexpr int HALF = Geo<D>::DPAD / 2;
     const int64_t q = (int64_t)blockIdx.x * 128 + threadIdx.x;
     const int h = blockIdx.y;
-    if (q >= a.nq) return;
-    const int64_t qt = q / 128;
-    const int rr = (int)(q % 128);
-    float g[D], x[D];
+    const bool live = q < a.nq;
+    const bool want_pg = a.dgain_q != nullptr || a.dbase != nullptr;
+    float pg[D], pb[3] = {0.f, 0.f, 0.f};  // parameter-gradient partials of this row
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-        const float4 *src =
-            reinterpret_cast<const float4 *>(a.dqacc + ((((size_t)h * a.nqt + qt) * 2 + hf) * 128 + rr) * HALF);
+    for (int d = 0; d < D; ++d) pg[d] = 0.f;
+    if (live) {
+        const int64_t qt = q / 128;
+        const int rr = (int)(q % 128);
+        float g[D], x[D];
 #pragma unroll
-        for (int c = 0; c < HALF / 4; ++c) {
-            if (hf * HALF + 4 * c < D) {
-                const float4 f = src[c];
-                g[hf * HALF + 4 * c] = f.x;
-                g[hf * HALF + 4 * c + 1] = f.y;
-                g[hf * HALF + 4 * c + 2] = f.z;
-                g[hf * HALF + 4 * c + 3] = f.w;
+        for (int hf = 0; hf < 2; ++hf) {
+            const float4 *src =
+                reinterpret_cast<const float4 *>(a.dqacc + ((((size_t)h * a.nqt + qt) * 2 + hf) * 128 + rr) * HALF);
+#pragma unroll
+            for (int c = 0; c < HALF / 4; ++c) {
+                if (hf * HALF + 4 * c < D) {
+                    const float4 f = src[c];
+                    g[hf * HALF + 4 * c] = f.x;
+                    g[hf * HALF + 4 * c + 1] = f.y;
+                    g[hf * HALF + 4 * c + 2] = f.z;
+                    g[hf * HALF + 4 * c + 3] = f.w;
+                }
+            }
+        }
+        const float sc = a.scale / ds_scale(a.bounds);
+#pragma unroll
+        for (int d = 0; d < D; ++d) g[d] *= sc;
+        const size_t row = (size_t)q * a.hq + h;
+        load_row_bf16<D>(a.q + row * D, x);
+        if (want_pg)
+            qk_param_grads<D>(x, g, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps, a.coef, pg,
+                              pb);
+        qk_prologue_bwd<D>(x, g, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps);
+        float4 *dst = reinterpret_cast<float4 *>(a.dq + row * D);
+#pragma unroll
+        for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(g[4 * c], g[4 * c + 1], g[4 * c + 2], g[4 * c + 3]);
+    }
+    if (want_pg) {
+        // the block's 128 rows: warp sums, then one add per value for the block
+        __shared__ float red[4][D + 3];
+#pragma unroll
+        for (int d = 0; d < D; ++d)
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) pg[d] += __shfl_xor_sync(0xffffffffu, pg[d], o);
+#pragma unroll
+        for (int e = 0; e < 3; ++e)
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) pb[e] += __shfl_xor_sync(0xffffffffu, pb[e], o);
+        const int w = threadIdx.x / 32;
+        if ((threadIdx.x & 31) == 0) {
+#pragma unroll
+            for (int d = 0; d < D; ++d) red[w][d] = pg[d];
+#pragma unroll
+            for (int e = 0; e < 3; ++e) red[w][D + e] = pb[e];
+        }
+        __syncthreads();
+        const int t = threadIdx.x;
+        if (t < D + 3) {
+            const float v = red[0][t] + red[1][t] + red[2][t] + red[3][t];
+            if (t < D) {
+                if (a.dgain_q) atomicAdd(a.dgain_q + t, v);
+            } else if (a.dbase) {
+                atomicAdd(a.dbase + (t - D), v);
             }
         }
     }
-    const float sc = a.scale / ds_scale(a.bounds);
-#pragma unroll
-    for (int d = 0; d < D; ++d) g[d] *= sc;
-    const size_t row = (size_t)q * a.hq + h;
-    load_row_bf16<D>(a.q + row * D, x);
-    qk_prologue_bwd<D>(x, g, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps);
-    float4 *dst = reinterpret_cast<float4 *>(a.dq + row * D);
-#pragma unroll
-    for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(g[4 * c], g[4 * c + 1], g[4 * c + 2], g[4 * c + 3]);
 }
 
 template <int D>
@@ -780,6 +852,11 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     auto *dqacc = reinterpret_cast<float *>(ws + 2 * kvb + 2 * qb + 2 * vb + 256);
     if (cudaMemsetAsync(bounds, 0, 2 * sizeof(float), stream) != cudaSuccess) return BCA_ERR_CUDA;
     if (cudaMemsetAsync(dqacc, 0, dq_acc_bytes(P), stream) != cudaSuccess) return BCA_ERR_CUDA;
+    // parameter gradients are sums over rows: start them at zero
+    if (io.dq_gain && cudaMemsetAsync(io.dq_gain, 0, D * sizeof(float), stream) != cudaSuccess) return BCA_ERR_CUDA;
+    if (io.dk_gain && cudaMemsetAsync(io.dk_gain, 0, D * sizeof(float), stream) != cudaSuccess) return BCA_ERR_CUDA;
+    if (io.drope_base && cudaMemsetAsync(io.drope_base, 0, 3 * sizeof(float), stream) != cudaSuccess)
+        return BCA_ERR_CUDA;
 
     PrepArgs pa;
     pa.q = static_cast<const __nv_bfloat16 *>(io.q);
@@ -875,6 +952,9 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     ba.dv = io.dv;
     ba.dkc = io.dk_cache;
     ba.dvc = io.dv_cache;
+    ba.dgain_k = io.dk_gain;
+    ba.dbase = io.drope_base;
+    for (int i = 0; i < 24; ++i) ba.coef[i] = P.rope_base_coef[i];
     ba.status = P.d_status;
     if (cudaFuncSetAttribute(bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES) != cudaSuccess)
         return BCA_ERR_CUDA;
@@ -900,6 +980,9 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     da.dq = io.dq;
     da.dqacc = dqacc;
     da.bounds = bounds;
+    da.dgain_q = io.dq_gain;
+    da.dbase = io.drope_base;
+    for (int i = 0; i < 24; ++i) da.coef[i] = P.rope_base_coef[i];
     {
         ProfScope ps(P, BCA_KERNEL_BWD_DQ, stream);
         if (P.nq > 0) bwd_dq_kernel<D><<<dim3((unsigned)P.nqt, (unsigned)P.hq), 128, 0, stream>>>(da);

@@ -26,6 +26,7 @@ struct BwdIO {
     const void *dout;
     float *dq, *dk, *dv, *dk_cache, *dv_cache;
     void *workspace;
+    float *dq_gain, *dk_gain, *drope_base;  // optional parameter gradients (NULL = not wanted)
 };
 
 // Bytes of each K-hat / V image (all KV heads, all k-tiles), 256-byte rounded.

@@ -321,6 +321,11 @@ int compile_plan(Plan &P) {
             }
         }
     }
+    for (int a = 0; a < 3; ++a)
+        for (int k = 0; k < pairs && k < 8; ++k) {
+            const double e = -(double)k / (double)pairs;
+            P.rope_base_coef[8 * a + k] = (float)(e * std::pow((double)P.base[a], e - 1.0));
+        }
     return BCA_OK;
 }
 

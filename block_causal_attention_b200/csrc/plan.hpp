@@ -57,6 +57,8 @@ struct Plan {
     std::vector<float> rope;         // (cos, sin) pairs: [(axis_off[a] + p) * pairs + k]
     int32_t rope_axis_off[3] = {0, 0, 0};
     int32_t rope_pairs = 0;
+    // d(base_a^(-k/pairs))/d(base_a) at [8 a + k], for the gradient of the RoPE bases
+    float rope_base_coef[24] = {};
 
     // device copies (owned)
     int device = -1;

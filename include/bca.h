@@ -192,6 +192,21 @@ int bca_bwd(bca_plan_t plan, const void *q, const void *k, const void *v,
             float *dq, float *dk, float *dv, float *dk_cache, float *dv_cache,
             void *workspace, void *stream);
 
+/* bca_bwd plus the gradients of the prologue's parameters (MAGI-1 research notes,
+ * "Autoregressive denoising DiT": QK-Norm, and 3D RoPE with a learnable base frequency):
+ *   dq_gain    : fp32 [D], dL/d(q_gain), summed over every query row and head;
+ *   dk_gain    : fp32 [D], dL/d(k_gain), summed over every new key row and KV head (cache
+ *                keys are given post-prologue, so they do not depend on the gain);
+ *   drope_base : fp32 [3], dL/d(rope_base[t, h, w]), summed over Q and new K rows.
+ * Any of the three may be NULL (not computed); non-NULL ones are overwritten (4-byte
+ * aligned).  The sums are formed with atomic adds, so their last bits may differ between
+ * runs.  Everything else is as bca_bwd, which is this call with the three set to NULL. */
+int bca_bwd_ex(bca_plan_t plan, const void *q, const void *k, const void *v,
+               const void *k_cache, const void *v_cache, const float *q_gain,
+               const float *k_gain, const void *o, const float *lse, const void *dout,
+               float *dq, float *dk, float *dv, float *dk_cache, float *dv_cache,
+               float *dq_gain, float *dk_gain, float *drope_base, void *workspace, void *stream);
+
 /* Kernel kinds for per-kernel timing */
 #define BCA_KERNEL_KV_IMAGE 0      /* K-hat prologue + K/V tile images */
 #define BCA_KERNEL_FWD 1           /* attention forward */

@@ -93,6 +93,38 @@ def test_bwd_with_gains_random_slices_and_empty_rows():
             _err("dk_cache", dkc, rkc); _err("dv_cache", dvc, rvc)
 
 
+@pytest.mark.parametrize("name", ["tiny", "b45_replica", "p720_replica", "kvrange_replica"])
+def test_bwd_parameter_gradients(name):
+    """Gradients of the QK-Norm gains and the RoPE bases (bca_bwd_ex) against the oracle.
+    They are sums over every row and head, so they are compared relative to the largest
+    reference entry: max-abs error <= 1e-2 x max|ref| (the per-element dQ / dK tolerance
+    of 1e-2 relative to |dq| ~ 1 carried over to the sums); the ordinary gradients of the
+    same call must still meet their own tolerances."""
+    w = W.WORKLOADS[name]
+    x = W.make_inputs(w, "cuda", with_grad=True)
+    gen = torch.Generator().manual_seed(77)
+    qg = (0.5 + torch.rand(w.d, generator=gen)).float()
+    kg = (0.5 + torch.rand(w.d, generator=gen)).float()
+    p = Plan.from_workload(w)
+    o, lse = p.fwd(x["q"], x["k"], x["v"], x["k_cache"], x["v_cache"], q_gain=qg.cuda(), k_gain=kg.cuda())
+    out = p.bwd(x["q"], x["k"], x["v"], x["k_cache"], x["v_cache"], o, lse, x["do"], q_gain=qg.cuda(),
+                k_gain=kg.cuda(), param_grads=True)
+    torch.cuda.synchronize()
+    assert p.status() == _abi.BCA_OK
+    c = {k: (None if t is None else t.cpu()) for k, t in x.items()}
+    ref = oracle.backward(c["q"], c["k"], c["v"], c["k_cache"], c["v_cache"], c["do"], w.videos_array(),
+                          w.slices_array(), w.hq, w.hkv, base=w.rope_base, eps=w.eps, q_gain=qg.double().numpy(),
+                          k_gain=kg.double().numpy(), param_grads=True)
+    _err("dq", out[0], ref[0]); _err("dk", out[1], ref[1]); _err("dv", out[2], ref[2])
+    msgs = []
+    for nm, got, want in (("dq_gain", out[5], ref[7]), ("dk_gain", out[6], ref[8]), ("drope_base", out[7], ref[9])):
+        e = np.abs(got.double().cpu().numpy() - want).max()
+        scale = np.abs(want).max()
+        msgs.append(f"{nm}: max err {e:.3e} of max|ref| {scale:.3e}")
+        assert e <= 1e-2 * scale, msgs[-1]
+    print(name, "; ".join(msgs))
+
+
 @pytest.mark.parametrize("name", ["tiny", "b45_replica"])
 def test_bwd_large_upstream_gradient(name):
     """dO scaled by 2^12 (exact in bf16) pushes the bound 2 max|dO| max|v| on |dS| past
