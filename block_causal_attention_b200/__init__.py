@@ -51,6 +51,15 @@ class Plan:
         return cls(w.hq, w.hkv, w.d, w.videos_array(), w.num_cache_keys, w.slices_array(),
                    w.rope_base, w.eps, w.o_fp32 if o_fp32 is None else o_fp32, host_only)
 
+    def update_positions(self, videos, stream=None) -> None:
+        """Move the videos' start frames (t0) of this plan, same geometry otherwise: only the
+        RoPE positions and tables are rewritten (a sliding inference window)."""
+        import numpy as np
+        vid = np.ascontiguousarray(np.asarray(videos, dtype=np.int32).reshape(-1, 5))
+        st = None if self.host_only else self._stream(stream)
+        rc = self._lib.bca_plan_update_positions(self._h, vid.ctypes.data if len(vid) else None, len(vid), st)
+        _abi.check(rc, "bca_plan_update_positions")
+
     # ------------------------------------------------------------------ host
     def info(self) -> dict:
         inf = _abi.bca_plan_info()

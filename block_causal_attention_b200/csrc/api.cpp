@@ -82,7 +82,10 @@ int upload(bca::Plan &P) {
         !P.d_col_runs || !P.d_bwd_items)
         return BCA_ERR_CUDA;
     if (cudaMemset(P.d_status, 0, sizeof(int)) != cudaSuccess) return BCA_ERR_CUDA;
-    return BCA_OK;
+    P.rope_capacity = P.rope.size();
+    int rc = prepare_fwd(P);
+    if (rc == BCA_OK) rc = prepare_bwd(P);
+    return rc;
 }
 
 int check_device(const bca::Plan &P) {
@@ -116,6 +119,51 @@ int bca_plan_create(const bca_problem *problem, bca_plan_t *out) {
         return rc;
     }
     *out = h;
+    return BCA_OK;
+}
+
+int bca_plan_update_positions(bca_plan_t plan, const bca_video *videos, int num_videos, void *stream) {
+    if (!plan || num_videos < 0 || (num_videos > 0 && !videos)) return BCA_ERR_INVALID_ARGUMENT;
+    bca::Plan &P = plan->plan;
+    if ((size_t)num_videos != P.videos.size()) return BCA_ERR_INVALID_ARGUMENT;
+    for (int i = 0; i < num_videos; ++i) {
+        const bca_video &a = videos[i], &b = P.videos[i];
+        if (a.num_chunks != b.num_chunks || a.frames != b.frames || a.height != b.height || a.width != b.width)
+            return BCA_ERR_INVALID_ARGUMENT;
+        if (a.t0 < 0 || (int64_t)a.t0 + (int64_t)a.num_chunks * a.frames > INT32_MAX) return BCA_ERR_INVALID_ARGUMENT;
+    }
+    const bool on_device = !(P.flags & BCA_PLAN_HOST_ONLY);
+    if (on_device) {
+        int rc = check_device(P);
+        if (rc != BCA_OK) return rc;
+    }
+    bca::Plan next;  // positions only: build into a scratch plan, then commit
+    next.videos.assign(videos, videos + num_videos);
+    next.nq = P.nq;
+    next.d = P.d;
+    for (int a = 0; a < 3; ++a) next.base[a] = P.base[a];
+    int rc;
+    try {
+        rc = bca::build_positions(next);
+    } catch (const std::bad_alloc &) {
+        rc = BCA_ERR_NO_MEMORY;
+    }
+    if (rc != BCA_OK) return rc;
+    if (on_device && next.rope.size() > P.rope_capacity) return BCA_ERR_UNSUPPORTED;  // the t range grew
+    if (on_device) {
+        cudaStream_t s = static_cast<cudaStream_t>(stream);
+        // pageable sources: the copies are staged before return, ordered on the stream
+        if (cudaMemcpyAsync(const_cast<uint32_t *>(P.d_pos), next.pos.data(), next.pos.size() * sizeof(uint32_t),
+                            cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(const_cast<float *>(P.d_rope), next.rope.data(), next.rope.size() * sizeof(float),
+                            cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return BCA_ERR_CUDA;
+    }
+    P.videos.swap(next.videos);
+    P.pos.swap(next.pos);
+    P.rope.swap(next.rope);
+    P.rope_tbase = next.rope_tbase;
+    for (int a = 0; a < 3; ++a) P.rope_axis_off[a] = next.rope_axis_off[a];
     return BCA_OK;
 }
 

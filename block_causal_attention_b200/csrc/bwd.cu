@@ -956,8 +956,6 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     ba.dbase = io.drope_base;
     for (int i = 0; i < 24; ++i) ba.coef[i] = P.rope_base_coef[i];
     ba.status = P.d_status;
-    if (cudaFuncSetAttribute(bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES) != cudaSuccess)
-        return BCA_ERR_CUDA;
     {
         ProfScope ps(P, BCA_KERNEL_BWD, stream);
         bwd_kernel<D><<<(unsigned)P.bwd_items.size(), 384, L::BYTES, stream>>>(ba);
@@ -1008,6 +1006,21 @@ size_t dq_acc_bytes(const Plan &P) { return (size_t)P.hq * (size_t)P.nqt * 128 *
 
 size_t bwd_workspace_bytes(const Plan &P) {
     return 2 * kv_image_bytes(P) + 2 * q_image_bytes(P) + 2 * q_vector_bytes(P) + 256 + dq_acc_bytes(P);
+}
+
+// Shared-memory attribute of the backward kernel, set once per plan (see prepare_fwd).
+int prepare_bwd(const Plan &P) {
+    auto set = [](const void *f, int bytes) {
+        return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+    };
+    bool ok = true;
+    switch (P.d) {
+        case 24: ok = set((const void *)bwd_kernel<24>, BwdSmem<24>::BYTES); break;
+        case 32: ok = set((const void *)bwd_kernel<32>, BwdSmem<32>::BYTES); break;
+        case 48: ok = set((const void *)bwd_kernel<48>, BwdSmem<48>::BYTES); break;
+        default: return BCA_ERR_UNSUPPORTED;
+    }
+    return ok ? BCA_OK : BCA_ERR_CUDA;
 }
 
 int launch_bwd(Plan &P, const BwdIO &io, cudaStream_t stream) {

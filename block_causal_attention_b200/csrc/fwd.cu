@@ -552,8 +552,6 @@ int launch_fwd_d(Plan &P, const FwdIO &io, cudaStream_t stream) {
     fa.status = P.d_status;
     fa.timeout_ns = (P.flags & BCA_TEST_FORCE_TIMEOUT) ? 1000000ull : kWaitTimeoutNs;
     fa.skip_loads = (P.flags & BCA_TEST_FORCE_TIMEOUT) ? 1 : 0;
-    if (cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES) != cudaSuccess)
-        return BCA_ERR_CUDA;
     {
         ProfScope ps(P, BCA_KERNEL_FWD, stream);
         fwd_kernel<D><<<(unsigned)P.items.size(), 384, L::BYTES, stream>>>(fa);
@@ -570,6 +568,23 @@ size_t kv_image_bytes(const Plan &P) {
 }
 
 size_t fwd_workspace_bytes(const Plan &P) { return 2 * kv_image_bytes(P); }
+
+// The attention kernel needs more than 48 KB of dynamic shared memory; the attribute
+// is set once per plan (at creation, on the plan's device) so that no launch path makes
+// a non-stream call (launches stay capturable into CUDA graphs).
+int prepare_fwd(const Plan &P) {
+    auto set = [](const void *f, int bytes) {
+        return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+    };
+    bool ok = true;
+    switch (P.d) {
+        case 24: ok = set((const void *)fwd_kernel<24>, FwdSmem<24>::BYTES); break;
+        case 32: ok = set((const void *)fwd_kernel<32>, FwdSmem<32>::BYTES); break;
+        case 48: ok = set((const void *)fwd_kernel<48>, FwdSmem<48>::BYTES); break;
+        default: return BCA_ERR_UNSUPPORTED;
+    }
+    return ok ? BCA_OK : BCA_ERR_CUDA;
+}
 
 int launch_fwd(Plan &P, const FwdIO &io, cudaStream_t stream) {
     if (P.nq == 0) return BCA_OK;

@@ -40,6 +40,10 @@ size_t q_vector_bytes(const Plan &plan);
 size_t dq_acc_bytes(const Plan &plan);
 size_t bwd_workspace_bytes(const Plan &plan);
 
+// One-time per-plan kernel attributes (dynamic shared memory), on the plan's device.
+int prepare_fwd(const Plan &plan);
+int prepare_bwd(const Plan &plan);
+
 // Bracket a launch with events when the plan is profiling (no-op otherwise).
 struct ProfScope {
     Plan &plan;

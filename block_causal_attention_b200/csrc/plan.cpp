@@ -146,9 +146,9 @@ int validate_problem(const bca_problem *p, Plan &P) {
     for (const bca_video &v : P.videos) {
         if (v.num_chunks < 0 || v.frames <= 0 || v.height <= 0 || v.width <= 0 || v.t0 < 0)
             return BCA_ERR_INVALID_ARGUMENT;
-        // packed RoPE positions: t < 65536, h, w < 256
+        // packed RoPE positions: t - (smallest t0) < 65536, h, w < 256
         if (v.height > 256 || v.width > 256) return BCA_ERR_UNSUPPORTED;
-        if ((int64_t)v.t0 + (int64_t)v.num_chunks * v.frames > 65536) return BCA_ERR_UNSUPPORTED;
+        if ((int64_t)v.t0 + (int64_t)v.num_chunks * v.frames > INT32_MAX) return BCA_ERR_UNSUPPORTED;
         nq += (int64_t)v.num_chunks * v.frames * v.height * v.width;
     }
     P.nq = nq;
@@ -288,8 +288,19 @@ int compile_plan(Plan &P) {
         return x.head0 < y.head0;
     });
 
-    // ---- positions and RoPE tables ----
+    return build_positions(P);
+}
+
+// Packed positions of the new tokens and the RoPE cos/sin tables, from P.videos.  The
+// t field holds t - tbase (tbase = the smallest t0 of a non-empty video) and the t table
+// covers [tbase, tbase + extent), so a window that slides by shifting every t0 keeps
+// the same table size (bca_plan_update_positions relies on that).
+int build_positions(Plan &P) {
     P.pos.resize(P.nq);
+    int32_t tbase = INT32_MAX;
+    for (const bca_video &v : P.videos)
+        if (v.num_chunks > 0) tbase = std::min(tbase, v.t0);
+    if (tbase == INT32_MAX) tbase = 0;
     int32_t tmax = 0, hmax = 0, wmax = 0;
     int64_t n = 0;
     for (const bca_video &v : P.videos) {
@@ -297,7 +308,9 @@ int compile_plan(Plan &P) {
             for (int f = 0; f < v.frames; ++f)
                 for (int y = 0; y < v.height; ++y)
                     for (int x = 0; x < v.width; ++x) {
-                        const uint32_t t = (uint32_t)(v.t0 + c * v.frames + f);
+                        const int64_t trel = (int64_t)v.t0 + (int64_t)c * v.frames + f - tbase;
+                        if (trel >= 65536) return BCA_ERR_UNSUPPORTED;
+                        const uint32_t t = (uint32_t)trel;
                         P.pos[n++] = (t << 16) | ((uint32_t)y << 8) | (uint32_t)x;
                         tmax = std::max<int32_t>(tmax, (int32_t)t);
                         hmax = std::max(hmax, y);
@@ -306,6 +319,7 @@ int compile_plan(Plan &P) {
     }
     const int pairs = (P.d / 2) / 3;
     P.rope_pairs = pairs;
+    P.rope_tbase = tbase;
     const int32_t ext[3] = {tmax + 1, hmax + 1, wmax + 1};
     P.rope_axis_off[0] = 0;
     P.rope_axis_off[1] = ext[0];
@@ -313,8 +327,9 @@ int compile_plan(Plan &P) {
     P.rope.assign((size_t)(ext[0] + ext[1] + ext[2]) * pairs * 2, 0.0f);
     for (int a = 0; a < 3; ++a) {
         for (int32_t pp = 0; pp < ext[a]; ++pp) {
+            const double position = (double)pp + (a == 0 ? (double)tbase : 0.0);
             for (int k = 0; k < pairs; ++k) {
-                const double ang = (double)pp * std::pow((double)P.base[a], -(double)k / (double)pairs);
+                const double ang = position * std::pow((double)P.base[a], -(double)k / (double)pairs);
                 const size_t at = ((size_t)(P.rope_axis_off[a] + pp) * pairs + k) * 2;
                 P.rope[at] = (float)std::cos(ang);
                 P.rope[at + 1] = (float)std::sin(ang);

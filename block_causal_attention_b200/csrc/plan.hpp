@@ -57,6 +57,8 @@ struct Plan {
     std::vector<float> rope;         // (cos, sin) pairs: [(axis_off[a] + p) * pairs + k]
     int32_t rope_axis_off[3] = {0, 0, 0};
     int32_t rope_pairs = 0;
+    int32_t rope_tbase = 0;           // the t table starts at this absolute frame
+    size_t rope_capacity = 0;         // floats of the device RoPE table (set at upload)
     // d(base_a^(-k/pairs))/d(base_a) at [8 a + k], for the gradient of the RoPE bases
     float rope_base_coef[24] = {};
 
@@ -87,6 +89,9 @@ struct Plan {
 int validate_problem(const bca_problem *p, Plan &plan);
 // Compile the mask into runs / bitmasks, build the item schedule and the tables.
 int compile_plan(Plan &plan);
+// Positions and RoPE tables from plan.videos (part of compile_plan; also used when only
+// the videos' start frames change).
+int build_positions(Plan &plan);
 // Expand compiled tiles of rows [r0, r1) into a coverage map (host).
 int expand_rows(const Plan &plan, int64_t r0, int64_t r1, uint8_t *out);
 // Same from the transposed (backward) runs, for keys [k0, k1): out[(j - k0) * nq + i].

@@ -142,6 +142,18 @@ int bca_plan_expand_rows(bca_plan_t plan, int64_t row_begin, int64_t row_end, ui
  * out[(j - key_begin) * Nq + i].  Host only. */
 int bca_plan_expand_cols(bca_plan_t plan, int64_t key_begin, int64_t key_end, uint8_t *out);
 
+/* Streaming reuse of a plan (MAGI-1 research notes, "Inference tricks > KV Cache": the
+ * denoising window slides one chunk at a time).  Replace the plan's videos by `videos`
+ * that differ only in t0 (same count, chunks, frames, height, width): the mask, tiles and
+ * work items are unchanged and only the new tokens' positions and RoPE tables are
+ * rewritten (cudaMemcpyAsync on `stream`, after any launch already queued there; the
+ * host arguments may be freed on return).  Tables are stored relative to the smallest t0,
+ * so shifting every t0 by the same amount keeps their size; a change that would enlarge
+ * the t range returns BCA_ERR_UNSUPPORTED and changes nothing.  Launches captured in a
+ * CUDA graph keep working: they read the rewritten tables in place.  Returns
+ * BCA_ERR_INVALID_ARGUMENT for a changed geometry or a negative t0. */
+int bca_plan_update_positions(bca_plan_t plan, const bca_video *videos, int num_videos, void *stream);
+
 /* Bytes of caller-provided device workspace a pass needs (16-byte aligned). */
 size_t bca_workspace_bytes(bca_plan_t plan, int pass);
 
