@@ -104,6 +104,7 @@ struct BwdArgs {
     float *dk, *dv, *dkc, *dvc;
     float *dgain_k, *dbase;  // optional parameter gradients (K gain; RoPE bases, shared with Q)
     float coef[24];          // d(base_a^(-k/P))/d(base_a) at [8 a + k]
+    int32_t tbase;           // absolute frame of packed t = 0
     int *status;
 };
 
@@ -121,6 +122,7 @@ struct DqArgs {
     float *dq;
     float *dgain_q, *dbase;  // optional parameter gradients (Q gain; RoPE bases, shared with K)
     float coef[24];
+    int32_t tbase;
 };
 
 // Power-of-two scale sc applied to dS before its fp16 rounding: 1 unless the bound
@@ -736,7 +738,7 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                     load_row_bf16<D>(a.k + ((size_t)nn * a.hkv + g) * D, x);
                     if (want_pg)
                         qk_param_grads<D>(x, gk, __ldg(a.pos + nn), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps,
-                                          a.coef, pg, pb);
+                                          a.coef, a.tbase, pg, pb);
                     qk_prologue_bwd<D>(x, gk, __ldg(a.pos + nn), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps);
                     dst = a.dk + ((size_t)nn * a.hkv + g) * D;
                 }
@@ -796,8 +798,8 @@ __global__ void __launch_bounds__(128) bwd_dq_kernel(DqArgs a) {
         const size_t row = (size_t)q * a.hq + h;
         load_row_bf16<D>(a.q + row * D, x);
         if (want_pg)
-            qk_param_grads<D>(x, g, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps, a.coef, pg,
-                              pb);
+            qk_param_grads<D>(x, g, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps, a.coef,
+                              a.tbase, pg, pb);
         qk_prologue_bwd<D>(x, g, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps);
         float4 *dst = reinterpret_cast<float4 *>(a.dq + row * D);
 #pragma unroll
@@ -955,6 +957,7 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     ba.dgain_k = io.dk_gain;
     ba.dbase = io.drope_base;
     for (int i = 0; i < 24; ++i) ba.coef[i] = P.rope_base_coef[i];
+    ba.tbase = P.rope_tbase;
     ba.status = P.d_status;
     {
         ProfScope ps(P, BCA_KERNEL_BWD, stream);
@@ -981,6 +984,7 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     da.dgain_q = io.dq_gain;
     da.dbase = io.drope_base;
     for (int i = 0; i < 24; ++i) da.coef[i] = P.rope_base_coef[i];
+    da.tbase = P.rope_tbase;
     {
         ProfScope ps(P, BCA_KERNEL_BWD_DQ, stream);
         if (P.nq > 0) bwd_dq_kernel<D><<<dim3((unsigned)P.nqt, (unsigned)P.hq), 128, 0, stream>>>(da);

@@ -127,11 +127,12 @@ __device__ __forceinline__ void qk_prologue_bwd(const float (&x)[D], float (&g)[
 //   dg_d += (R^T dy)_d z_d;
 //   for pair k of axis a: dL/dangle = dy1 y0 - dy0 y1, and angle = pos_a base_a^(-k/P), so
 //   db_a += dL/dangle * pos_a * coef[8 a + k] with coef[8 a + k] = d(base_a^(-k/P))/d(base_a).
+// The packed t is relative to the plan's first frame tbase; pos_t = t + tbase.
 template <int D>
 __device__ __forceinline__ void qk_param_grads(const float (&x)[D], const float (&dy)[D], uint32_t pos,
                                                const float *gain, const float *rope, int32_t off0, int32_t off1,
-                                               int32_t off2, float eps, const float *coef, float (&dg)[D],
-                                               float (&db)[3]) {
+                                               int32_t off2, float eps, const float *coef, int32_t tbase,
+                                               float (&dg)[D], float (&db)[3]) {
     constexpr int P = Geo<D>::PAIRS;
     float ss = 0.f;
 #pragma unroll
@@ -141,6 +142,7 @@ __device__ __forceinline__ void qk_param_grads(const float (&x)[D], const float 
     for (int d = 6 * P; d < D; ++d) dg[d] = fmaf(dy[d], x[d] * r, dg[d]);  // channels RoPE leaves alone
     const int32_t p[3] = {(int32_t)(pos >> 16), (int32_t)((pos >> 8) & 255u), (int32_t)(pos & 255u)};
     const int32_t off[3] = {off0, off1, off2};
+    const float pabs[3] = {(float)(p[0] + tbase), (float)p[1], (float)p[2]};
 #pragma unroll
     for (int a = 0; a < 3; ++a) {
         const float2 *tab = reinterpret_cast<const float2 *>(rope) + (size_t)(off[a] + p[a]) * P;
@@ -152,7 +154,7 @@ __device__ __forceinline__ void qk_param_grads(const float (&x)[D], const float 
             const float h0 = z0 * (gain ? __ldg(gain + c0) : 1.0f), h1 = z1 * (gain ? __ldg(gain + c0 + 1) : 1.0f);
             const float y0 = h0 * cs.x - h1 * cs.y, y1 = h0 * cs.y + h1 * cs.x;
             const float dang = dy[c0 + 1] * y0 - dy[c0] * y1;
-            db[a] = fmaf(dang * (float)p[a], coef[8 * a + k], db[a]);
+            db[a] = fmaf(dang * pabs[a], coef[8 * a + k], db[a]);
             dg[c0] = fmaf(dy[c0] * cs.x + dy[c0 + 1] * cs.y, z0, dg[c0]);
             dg[c0 + 1] = fmaf(-dy[c0] * cs.y + dy[c0 + 1] * cs.x, z1, dg[c0 + 1]);
         }
