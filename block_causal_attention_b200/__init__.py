@@ -165,6 +165,26 @@ class Plan:
         _abi.check(rc, "bca_bwd_ex")
         return dq, dk, dv, dk_cache, dv_cache, dgq, dgk, dbase
 
+    def k_prologue(self, k, k_gain=None, *, out=None, stream=None):
+        """Post-prologue keys (bf16 [Nq, Hkv, D]) of the plan's new tokens."""
+        import torch
+        if out is None:
+            out = torch.empty((self.nq, self.hkv, self.d), device=k.device, dtype=torch.bfloat16)
+        _abi.check(self._lib.bca_k_prologue(self._h, _ptr(k), _ptr(k_gain), _ptr(out), self._stream(stream)),
+                   "bca_k_prologue")
+        return out
+
+    def k_prologue_bwd(self, k, dk_hat, k_gain=None, *, dk=None, accumulate=False, stream=None):
+        """dL/dk (fp32 [Nq, Hkv, D]) from dL/dk_hat through the prologue; added into dk
+        when accumulate=True."""
+        import torch
+        if dk is None:
+            dk = torch.zeros((self.nq, self.hkv, self.d), device=k.device, dtype=torch.float32)
+        _abi.check(self._lib.bca_k_prologue_bwd(self._h, _ptr(k), _ptr(k_gain), _ptr(dk_hat), _ptr(dk),
+                                                1 if accumulate else 0, self._stream(stream)),
+                   "bca_k_prologue_bwd")
+        return dk
+
     def profile(self, enable: bool = True) -> None:
         """Bracket every kernel launched for this plan with CUDA events."""
         _abi.check(self._lib.bca_profile_enable(self._h, 1 if enable else 0), "bca_profile_enable")

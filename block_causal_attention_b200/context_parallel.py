@@ -1,0 +1,331 @@
+"""Context parallelism: one block-causal attention problem spread over the ranks of a
+process group, by query chunk.
+
+The route of the pages (MAGI-1 research notes, "Infra > MagiAttention": the dispatch
+solver balances the unmasked area per rank, then key/value chunks are group-cast to the
+ranks whose queries see them and the gradients are group-reduced back; the Interview's
+answer on the dispatch solver gives the same cost model):
+
+1. dispatch: every chunk of every video goes to one rank, longest-first onto the least
+   loaded rank, where a chunk's load is its number of visible (query, key) pairs;
+2. each rank builds a local problem: its chunks are the new tokens (one single-chunk
+   video each, at the chunk's frames), the keys it needs from other ranks' tokens and
+   from the global cache become its cache (post-prologue keys), and every FULL slice is
+   cut into pieces that map contiguous global key ranges onto contiguous local ones;
+3. forward: each rank computes the post-prologue keys of its own tokens
+   (``k_prologue``) and one all-to-all-v sends the rows each other rank needs;
+4. backward: the local backward returns gradients for the borrowed rows as cache
+   gradients; a second all-to-all-v sends them to the owners, which add them (K through
+   ``k_prologue_bwd``); gradients of the global cache are summed over ranks.
+
+Every rank derives the whole dispatch from the same inputs, so no metadata is exchanged.
+Only FULL slices are handled (the slice language has no offset with which to cut a
+CAUSAL slice into shifted pieces); every workload of the pages is written with FULL
+slices.  The attention engine is pluggable: the default is this package's CUDA ``Plan``.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Callable, List, Optional, Sequence
+
+import numpy as np
+
+SLICE_FULL = 0
+
+
+@dataclasses.dataclass(frozen=True)
+class Chunk:
+    """One chunk of one video: new tokens [start, end) in the global token order."""
+    start: int
+    end: int
+    frames: int
+    height: int
+    width: int
+    t0: int  # first frame of the chunk
+
+
+def chunks_of(videos) -> List[Chunk]:
+    out = []
+    n = 0
+    for nc, f, h, w, t0 in np.asarray(videos, np.int64).reshape(-1, 5):
+        size = int(f * h * w)
+        for c in range(int(nc)):
+            out.append(Chunk(n, n + size, int(f), int(h), int(w), int(t0 + c * f)))
+            n += size
+    return out
+
+
+def _merge(iv):
+    iv = sorted(iv)
+    out = []
+    for a, b in iv:
+        if a >= b:
+            continue
+        if out and a <= out[-1][1]:
+            out[-1][1] = max(out[-1][1], b)
+        else:
+            out.append([a, b])
+    return [(a, b) for a, b in out]
+
+
+def chunk_rows(slices, chunk: Chunk, nc: int):
+    """Row groups of a chunk with their merged visible key intervals: a list of
+    (q_begin, q_end, [(k_begin, k_end), ...]) in global query / key indices."""
+    sl = np.asarray(slices, np.int64).reshape(-1, 5)
+    cuts = {chunk.start, chunk.end}
+    mine = []
+    for q0, q1, k0, k1, t in sl:
+        if t != SLICE_FULL:
+            raise NotImplementedError("context parallelism handles FULL slices only")
+        a, b = max(int(q0), chunk.start), min(int(q1), chunk.end)
+        if a < b and k0 < k1:
+            mine.append((a, b, int(k0), int(k1)))
+            cuts.update((a, b))
+    cuts = sorted(cuts)
+    groups = []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        iv = _merge([(k0, k1) for (s0, s1, k0, k1) in mine if s0 <= a and b <= s1])
+        if iv:
+            groups.append((a, b, iv))
+    return groups
+
+
+def chunk_area(slices, chunk: Chunk, nc: int) -> int:
+    return sum((b - a) * sum(k1 - k0 for k0, k1 in iv) for a, b, iv in chunk_rows(slices, chunk, nc))
+
+
+def dispatch(chunks: Sequence[Chunk], areas: Sequence[int], world: int) -> List[int]:
+    """Owner rank of each chunk: longest first onto the least loaded rank (ties: the
+    lower rank), so every rank computes the same answer."""
+    order = sorted(range(len(chunks)), key=lambda i: (-areas[i], i))
+    load = [0] * world
+    owner = [0] * len(chunks)
+    for i in order:
+        r = min(range(world), key=lambda x: (load[x], x))
+        owner[i] = r
+        load[r] += areas[i]
+    return owner
+
+
+@dataclasses.dataclass
+class LocalProblem:
+    rank: int
+    chunks: List[int]            # indices of this rank's chunks, in global order
+    tokens: np.ndarray           # global token index of each local new token
+    videos: np.ndarray           # [n_chunks, 5] single-chunk videos
+    cache_rows: np.ndarray       # global cache rows needed, sorted
+    remote_rows: np.ndarray      # global token indices of borrowed keys, sorted
+    slices: np.ndarray           # [m, 5] local FULL slices
+    area: int
+
+    @property
+    def num_cache_keys(self) -> int:
+        return len(self.cache_rows) + len(self.remote_rows)
+
+
+class ContextParallelPlan:
+    """The dispatch and the local problem of every rank, computed identically on all."""
+
+    def __init__(self, world: int, videos, num_cache_keys: int, slices):
+        self.world = int(world)
+        self.nc = int(num_cache_keys)
+        self.chunks = chunks_of(videos)
+        self.nq = self.chunks[-1].end if self.chunks else 0
+        self.rows = [chunk_rows(slices, c, self.nc) for c in self.chunks]
+        self.areas = [sum((b - a) * sum(k1 - k0 for k0, k1 in iv) for a, b, iv in g) for g in self.rows]
+        self.owner = dispatch(self.chunks, self.areas, self.world)
+        self.token_owner = np.zeros(self.nq, np.int64)
+        for c, r in zip(self.chunks, self.owner):
+            self.token_owner[c.start:c.end] = r
+        self.local = [self._local(r) for r in range(self.world)]
+        # exchange plan: rows[src][dst] = global tokens src sends to dst (in dst's order)
+        self.send_rows = [[np.zeros(0, np.int64) for _ in range(self.world)] for _ in range(self.world)]
+        for dst in range(self.world):
+            rr = self.local[dst].remote_rows
+            own = self.token_owner[rr] if len(rr) else np.zeros(0, np.int64)
+            for src in range(self.world):
+                self.send_rows[src][dst] = rr[own == src]
+
+    def _local(self, r: int) -> LocalProblem:
+        mine = [i for i, o in enumerate(self.owner) if o == r]
+        spans = [(self.chunks[i].start, self.chunks[i].end) for i in mine]
+        tokens = np.concatenate([np.arange(a, b) for a, b in spans]) if mine else np.zeros(0, np.int64)
+        first_local = np.cumsum([0] + [b - a for a, b in spans])
+        videos = np.asarray([[1, self.chunks[i].frames, self.chunks[i].height, self.chunks[i].width,
+                              self.chunks[i].t0] for i in mine], np.int32).reshape(-1, 5)
+        nk = self.nc + self.nq
+        own = np.zeros(nk, bool)
+        own[self.nc + tokens] = True
+        need = np.zeros(nk, bool)
+        for i in mine:
+            for a, b, iv in self.rows[i]:
+                for k0, k1 in iv:
+                    need[k0:k1] = True
+        need &= ~own
+        cache_rows = np.flatnonzero(need[:self.nc]).astype(np.int64)
+        remote_rows = np.flatnonzero(need[self.nc:]).astype(np.int64)
+        nc_loc = len(cache_rows) + len(remote_rows)
+        # global key -> local key: needed cache rows, then borrowed tokens, then own tokens
+        lk = np.full(nk, -1, np.int64)
+        lk[cache_rows] = np.arange(len(cache_rows))
+        lk[self.nc + remote_rows] = len(cache_rows) + np.arange(len(remote_rows))
+        lk[self.nc + tokens] = nc_loc + np.arange(len(tokens))
+        out = []
+        area = 0
+        for ci, i in enumerate(mine):
+            c = self.chunks[i]
+            for a, b, iv in self.rows[i]:
+                qa, qb = a - c.start + first_local[ci], b - c.start + first_local[ci]
+                for k0, k1 in iv:
+                    area += (b - a) * (k1 - k0)
+                    seg = lk[k0:k1]
+                    # pieces: maximal runs where the local index advances by one
+                    cuts = np.flatnonzero(np.diff(seg) != 1) + 1
+                    starts = np.concatenate([[0], cuts])
+                    ends = np.concatenate([cuts, [k1 - k0]])
+                    for s0, s1 in zip(starts, ends):
+                        out.append((qa, qb, int(seg[s0]), int(seg[s0]) + int(s1 - s0), SLICE_FULL))
+        sl = np.asarray(out, np.int64).reshape(-1, 5)
+        return LocalProblem(r, mine, tokens, videos, cache_rows, remote_rows, sl, area)
+
+
+# ----------------------------------------------------------------------------- runtime
+
+def _default_engine(hq, hkv, d, videos, num_cache_keys, slices, rope_base, eps, o_fp32):
+    from . import Plan
+    return Plan(hq, hkv, d, videos, num_cache_keys, slices, rope_base, eps, o_fp32)
+
+
+def _all_to_all_rows(group, send: List, recv_counts: List[int], row_shape, like):
+    """Rows of `send[dst]` go to rank dst; returns the received rows per source rank.
+    Rows are moved bit-exactly (as 16-bit integers for 16-bit types)."""
+    import torch
+    import torch.distributed as dist
+    world = len(send)
+    width = int(np.prod(row_shape))
+    flat = [s.reshape(-1, width) for s in send]
+    sbuf = torch.cat(flat, 0) if flat else like.new_zeros((0, width))
+    rbuf = like.new_empty((sum(recv_counts), width))
+    as_int = sbuf.dtype in (torch.bfloat16, torch.float16)
+    sview = sbuf.view(torch.int16) if as_int else sbuf
+    rview = rbuf.view(torch.int16) if as_int else rbuf
+    if world == 1:
+        rview.copy_(sview)
+    else:
+        dist.all_to_all_single(rview, sview, output_split_sizes=list(recv_counts),
+                               input_split_sizes=[int(f.shape[0]) for f in flat], group=group)
+    out, o = [], 0
+    for c in recv_counts:
+        out.append(rbuf[o:o + c].reshape((c,) + tuple(row_shape)))
+        o += c
+    return out
+
+
+class ContextParallelAttention:
+    """One rank's part of a context-parallel attention problem.  `q_local`, `k_local`,
+    `v_local`, `do_local` hold this rank's tokens (``local.tokens``); the cache is given
+    whole on every rank (post-prologue keys and values)."""
+
+    def __init__(self, group, rank: int, world: int, hq: int, hkv: int, d: int, videos, num_cache_keys: int,
+                 slices, rope_base=(1e4, 1e4, 1e4), eps: float = 1e-6, o_fp32: bool = False,
+                 engine: Optional[Callable] = None):
+        self.group, self.rank, self.world = group, int(rank), int(world)
+        self.hq, self.hkv, self.d = hq, hkv, d
+        self.cp = ContextParallelPlan(world, videos, num_cache_keys, slices)
+        self.local = self.cp.local[self.rank]
+        eng = engine or _default_engine
+        self.plan = eng(hq, hkv, d, self.local.videos, self.local.num_cache_keys, self.local.slices, rope_base,
+                        eps, o_fp32)
+        self._saved = None
+
+    def _gather_keys(self, khat_local, v_local):
+        """Rows of [K-hat | V] of this rank's tokens that the other ranks need, sent; the
+        borrowed rows received, in the order of local.remote_rows."""
+        import torch
+        cp, r = self.cp, self.rank
+        pos_in_local = {int(t): j for j, t in enumerate(self.local.tokens)}
+        kv = torch.stack([khat_local, v_local], 1)                      # [n, 2, Hkv, D]
+        send = []
+        for dst in range(self.world):
+            rows = cp.send_rows[r][dst]
+            idx = torch.as_tensor([pos_in_local[int(t)] for t in rows], dtype=torch.long, device=kv.device)
+            send.append(kv.index_select(0, idx))
+        recv_counts = [len(cp.send_rows[src][r]) for src in range(self.world)]
+        got = _all_to_all_rows(self.group, send, recv_counts, kv.shape[1:], kv)
+        # reorder to local.remote_rows: each source sent its subset in global order
+        rr = self.local.remote_rows
+        order = {}
+        for src in range(self.world):
+            for j, t in enumerate(cp.send_rows[src][r]):
+                order[int(t)] = (src, j)
+        if len(rr):
+            cat = torch.cat(got, 0)
+            offs = np.cumsum([0] + recv_counts)
+            idx = torch.as_tensor([offs[order[int(t)][0]] + order[int(t)][1] for t in rr], dtype=torch.long,
+                                  device=kv.device)
+            rem = cat.index_select(0, idx)
+        else:
+            rem = kv.new_zeros((0,) + tuple(kv.shape[1:]))
+        return rem[:, 0], rem[:, 1]
+
+    def _local_cache(self, k_cache, v_cache, rk, rv):
+        import torch
+        rows = torch.as_tensor(self.local.cache_rows, dtype=torch.long, device=rk.device)
+        if len(self.local.cache_rows):
+            kc, vc = k_cache.index_select(0, rows), v_cache.index_select(0, rows)
+            return torch.cat([kc, rk], 0), torch.cat([vc, rv], 0)
+        return rk, rv
+
+    def forward(self, q_local, k_local, v_local, k_cache=None, v_cache=None, q_gain=None, k_gain=None):
+        khat = self.plan.k_prologue(k_local, k_gain)
+        rk, rv = self._gather_keys(khat, v_local)
+        kc, vc = self._local_cache(k_cache, v_cache, rk, rv)
+        if self.local.num_cache_keys == 0:
+            kc = vc = None
+        o, lse = self.plan.fwd(q_local, k_local, v_local, kc, vc, q_gain=q_gain, k_gain=k_gain)
+        self._saved = (kc, vc)
+        return o, lse
+
+    def backward(self, q_local, k_local, v_local, k_cache, v_cache, o, lse, do_local, q_gain=None, k_gain=None):
+        """(dq, dk, dv) of this rank's tokens and (dk_cache, dv_cache) of the global cache
+        (summed over ranks, on every rank; None without a cache)."""
+        import torch
+        import torch.distributed as dist
+        kc, vc = self._saved
+        dq, dk, dv, dkc, dvc = self.plan.bwd(q_local, k_local, v_local, kc, vc, o, lse, do_local,
+                                             q_gain=q_gain, k_gain=k_gain)
+        ncl = len(self.local.cache_rows)
+        gk = gv = None
+        if self.cp.nc:
+            gk = dk.new_zeros((self.cp.nc, self.hkv, self.d))
+            gv = dk.new_zeros((self.cp.nc, self.hkv, self.d))
+            if ncl:
+                rows = torch.as_tensor(self.local.cache_rows, dtype=torch.long, device=dk.device)
+                gk.index_add_(0, rows, dkc[:ncl])
+                gv.index_add_(0, rows, dvc[:ncl])
+            if self.world > 1:
+                dist.all_reduce(gk, group=self.group)
+                dist.all_reduce(gv, group=self.group)
+        # borrowed rows' gradients go back to their owners
+        cp, r = self.cp, self.rank
+        rem_k = dkc[ncl:] if dkc is not None else dk.new_zeros((0, self.hkv, self.d))
+        rem_v = dvc[ncl:] if dvc is not None else dv.new_zeros((0, self.hkv, self.d))
+        grads = torch.stack([rem_k, rem_v], 1)                             # [n_remote, 2, Hkv, D]
+        rpos = {int(t): j for j, t in enumerate(self.local.remote_rows)}
+        send = []
+        for dst in range(self.world):
+            idx = torch.as_tensor([rpos[int(t)] for t in cp.send_rows[dst][r]], dtype=torch.long,
+                                  device=grads.device)
+            send.append(grads.index_select(0, idx))
+        recv_counts = [len(cp.send_rows[r][src]) for src in range(self.world)]
+        got = _all_to_all_rows(self.group, send, recv_counts, grads.shape[1:], grads)
+        pos_in_local = {int(t): j for j, t in enumerate(self.local.tokens)}
+        dkh = dk.new_zeros(dk.shape)
+        for src in range(self.world):
+            rows = cp.send_rows[r][src]
+            if len(rows):
+                idx = torch.as_tensor([pos_in_local[int(t)] for t in rows], dtype=torch.long, device=dk.device)
+                dkh.index_add_(0, idx, got[src][:, 0])
+                dv.index_add_(0, idx, got[src][:, 1])
+        dk = self.plan.k_prologue_bwd(k_local, dkh, k_gain, dk=dk, accumulate=True)
+        return dq, dk, dv, gk, gv

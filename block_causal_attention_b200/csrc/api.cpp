@@ -283,6 +283,30 @@ int bca_bwd(bca_plan_t plan, const void *q, const void *k, const void *v, const 
                       nullptr, nullptr, nullptr, workspace, stream);
 }
 
+int bca_k_prologue(bca_plan_t plan, const void *k, const float *k_gain, void *k_hat, void *stream) {
+    if (!plan) return BCA_ERR_INVALID_ARGUMENT;
+    bca::Plan &P = plan->plan;
+    int rc = check_device(P);
+    if (rc != BCA_OK) return rc;
+    if (P.nq == 0) return BCA_OK;
+    if (!k || !k_hat) return BCA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(k) || !aligned16(k_hat) || (k_gain && !aligned16(k_gain))) return BCA_ERR_MISALIGNED;
+    return bca::launch_k_prologue(P, k, k_gain, k_hat, static_cast<cudaStream_t>(stream));
+}
+
+int bca_k_prologue_bwd(bca_plan_t plan, const void *k, const float *k_gain, const float *dk_hat, float *dk,
+                       int accumulate, void *stream) {
+    if (!plan) return BCA_ERR_INVALID_ARGUMENT;
+    bca::Plan &P = plan->plan;
+    int rc = check_device(P);
+    if (rc != BCA_OK) return rc;
+    if (P.nq == 0) return BCA_OK;
+    if (!k || !dk_hat || !dk) return BCA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(k) || !aligned16(dk_hat) || !aligned16(dk) || (k_gain && !aligned16(k_gain)))
+        return BCA_ERR_MISALIGNED;
+    return bca::launch_k_prologue_bwd(P, k, k_gain, dk_hat, dk, accumulate, static_cast<cudaStream_t>(stream));
+}
+
 int bca_profile_enable(bca_plan_t plan, int enable) {
     if (!plan) return BCA_ERR_INVALID_ARGUMENT;
     drop_profile(plan->plan);

@@ -40,6 +40,12 @@ size_t q_vector_bytes(const Plan &plan);
 size_t dq_acc_bytes(const Plan &plan);
 size_t bwd_workspace_bytes(const Plan &plan);
 
+// K prologue over the plan's new tokens (bf16 K-hat rows) and its backward
+// (dk = or += J^T dk_hat), for context-parallel exchange of post-prologue keys.
+int launch_k_prologue(const Plan &plan, const void *k, const float *k_gain, void *k_hat, cudaStream_t stream);
+int launch_k_prologue_bwd(const Plan &plan, const void *k, const float *k_gain, const float *dk_hat, float *dk,
+                          int accumulate, cudaStream_t stream);
+
 // One-time per-plan kernel attributes (dynamic shared memory), on the plan's device.
 int prepare_fwd(const Plan &plan);
 int prepare_bwd(const Plan &plan);

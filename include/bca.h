@@ -219,6 +219,21 @@ int bca_bwd_ex(bca_plan_t plan, const void *q, const void *k, const void *v,
                float *dq, float *dk, float *dv, float *dk_cache, float *dv_cache,
                float *dq_gain, float *dk_gain, float *drope_base, void *workspace, void *stream);
 
+/* The key prologue of bca_fwd (QK-Norm + 3D RoPE at the plan's positions of its new
+ * tokens) as a stand-alone pass, and its backward.  Used by context parallelism: the
+ * rank that owns a token computes its post-prologue key once and sends it to the ranks
+ * whose queries see it (there it is a cache key); the gradients they return w.r.t. that
+ * key are mapped back through the prologue by the owner (MAGI-1 research notes,
+ * "Infra > MagiAttention": group-cast and group-reduce).
+ *   k      : bf16 [Nq][Hkv][D], the plan's new tokens' raw keys; k_gain: fp32 [D] or NULL;
+ *   k_hat  : bf16 [Nq][Hkv][D] out (RNE of the fp32 result);
+ *   dk_hat : fp32 [Nq][Hkv][D], dL/dk_hat;  dk: fp32 [Nq][Hkv][D] out, overwritten, or
+ *            added to when accumulate != 0.
+ * 16-byte aligned pointers; asynchronous on `stream`. */
+int bca_k_prologue(bca_plan_t plan, const void *k, const float *k_gain, void *k_hat, void *stream);
+int bca_k_prologue_bwd(bca_plan_t plan, const void *k, const float *k_gain, const float *dk_hat, float *dk,
+                       int accumulate, void *stream);
+
 /* Kernel kinds for per-kernel timing */
 #define BCA_KERNEL_KV_IMAGE 0      /* K-hat prologue + K/V tile images */
 #define BCA_KERNEL_FWD 1           /* attention forward */

@@ -1,0 +1,223 @@
+"""Context parallelism: dispatch and local problems (host), the exchange through
+torch.distributed with gloo ranks on CPU (attention by the fp64 oracle, injected as the
+engine), and the CUDA entry points it uses.  The N > 1 path cannot run on one GPU, so
+its collectives are exercised here with gloo."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_causal_attention_b200 import context_parallel as CP
+from block_causal_attention_b200 import workloads as W
+
+NAMES = ["tiny", "b45_replica", "packed_replica", "kvrange_replica", "p720_replica"]
+
+
+def _local_mask(cp, r):
+    """The rank's local mask mapped back to global (query token, global key) pairs."""
+    lp = cp.local[r]
+    nq_l, nc_l = len(lp.tokens), lp.num_cache_keys
+    m = oracle.mask_dense(lp.slices, nq_l, nc_l + nq_l)
+    key_of = np.concatenate([lp.cache_rows, cp.nc + lp.remote_rows, cp.nc + lp.tokens]).astype(np.int64)
+    g = np.zeros((cp.nq, cp.nc + cp.nq), bool)
+    qi, kj = np.nonzero(m)
+    g[lp.tokens[qi], key_of[kj]] = True
+    return g
+
+
+@pytest.mark.parametrize("name", NAMES)
+@pytest.mark.parametrize("world", [1, 2, 3, 4])
+def test_local_problems_reproduce_the_global_mask(name, world):
+    w = W.WORKLOADS[name]
+    cp = CP.ContextParallelPlan(world, w.videos_array(), w.num_cache_keys, w.slices_array())
+    ref = oracle.mask_dense(w.slices_array(), w.nq, w.nk).astype(bool)
+    union = np.zeros_like(ref)
+    for r in range(world):
+        lm = _local_mask(cp, r)
+        assert not (union & lm).any()                        # every query row has one owner
+        union |= lm
+        assert cp.local[r].area == int(lm.sum())
+    assert np.array_equal(union, ref)
+    assert sorted(np.concatenate([cp.local[r].tokens for r in range(world)]).tolist()) == list(range(w.nq))
+
+
+def test_dispatch_balances_area():
+    areas = [9, 7, 6, 5, 5, 4, 2, 1]
+    ch = [CP.Chunk(i, i + 1, 1, 1, 1, 0) for i in range(len(areas))]
+    owner = CP.dispatch(ch, areas, 3)
+    load = [sum(a for a, o in zip(areas, owner) if o == r) for r in range(3)]
+    assert max(load) - min(load) <= 1 and sum(load) == sum(areas)
+
+
+def test_causal_slices_are_rejected():
+    with pytest.raises(NotImplementedError):
+        CP.ContextParallelPlan(2, [[2, 1, 2, 2, 0]], 0, [[0, 8, 0, 8, 1]])
+
+
+# --------------------------------------------------------------------------- gloo ranks
+
+class OracleEngine:
+    """The attention engine on the fp64 oracle (test infrastructure only)."""
+
+    def __init__(self, hq, hkv, d, videos, nc, slices, base, eps, o_fp32):
+        self.hq, self.hkv, self.d = hq, hkv, d
+        self.videos, self.slices, self.base, self.eps = np.asarray(videos), np.asarray(slices), base, eps
+        self.pos = oracle.positions(self.videos) if len(self.videos) else np.zeros((0, 3), np.int32)
+
+    def k_prologue(self, k, k_gain=None):
+        return torch.from_numpy(oracle.prologue(k, self.pos, self.base, self.eps, k_gain))
+
+    def k_prologue_bwd(self, k, dk_hat, k_gain=None, dk=None, accumulate=False):
+        g = torch.from_numpy(oracle.prologue_bwd(k, self.pos, dk_hat, self.base, self.eps, k_gain))
+        return dk + g if accumulate else g
+
+    def fwd(self, q, k, v, kc, vc, q_gain=None, k_gain=None):
+        o, lse = oracle.forward(q, k, v, kc, vc, self.videos, self.slices, self.hq, self.hkv, base=self.base,
+                                eps=self.eps, q_gain=q_gain, k_gain=k_gain)
+        return torch.from_numpy(o), torch.from_numpy(lse)
+
+    def bwd(self, q, k, v, kc, vc, o, lse, do, q_gain=None, k_gain=None):
+        dq, dk, dv, dkc, dvc, _, _ = oracle.backward(q, k, v, kc, vc, do, self.videos, self.slices, self.hq,
+                                                     self.hkv, base=self.base, eps=self.eps, q_gain=q_gain,
+                                                     k_gain=k_gain)
+        t = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a))
+        return t(dq), t(dk), t(dv), t(dkc), t(dvc)
+
+
+def _small_cached():
+    """2 cached chunks + 3 query chunks of 16 tokens (1 x 4 x 4), block-causal over
+    (cache + queries): query chunk c sees the cache and query chunks 0..c."""
+    from types import SimpleNamespace
+    C, nc = 16, 32
+    sl = np.asarray([[C * c, C * (c + 1), 0, nc + C * (c + 1), 0] for c in range(3)], np.int64)
+    vid = np.asarray([[3, 1, 4, 4, 2]], np.int32)
+    return SimpleNamespace(nq=3 * C, nk=nc + 3 * C, hq=4, hkv=2, d=24, num_cache_keys=nc, rope_base=(50.0, 30.0, 20.0),
+                           eps=1e-6, videos_array=lambda: vid, slices_array=lambda: sl)
+
+
+def _workload(name):
+    return _small_cached() if name == "small_cached" else W.WORKLOADS[name]
+
+
+def _inputs(w):
+    g = torch.Generator().manual_seed(5)
+    r = lambda *s: torch.randn(*s, generator=g, dtype=torch.float64)
+    nc = w.num_cache_keys
+    x = {"q": r(w.nq, w.hq, w.d), "k": r(w.nq, w.hkv, w.d), "v": r(w.nq, w.hkv, w.d), "do": r(w.nq, w.hq, w.d),
+         "kc": r(nc, w.hkv, w.d) if nc else None, "vc": r(nc, w.hkv, w.d) if nc else None,
+         "qg": (0.5 + torch.rand(w.d, generator=g, dtype=torch.float64)),
+         "kg": (0.5 + torch.rand(w.d, generator=g, dtype=torch.float64))}
+    return x
+
+
+def _rank_main(rank, world, port, name, out_dir):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = _workload(name)
+        x = _inputs(w)
+        att = CP.ContextParallelAttention(None, rank, world, w.hq, w.hkv, w.d, w.videos_array(), w.num_cache_keys,
+                                          w.slices_array(), w.rope_base, w.eps, engine=OracleEngine)
+        tok = torch.as_tensor(att.local.tokens, dtype=torch.long)
+        ql, kl, vl, dol = (x[n].index_select(0, tok) for n in ("q", "k", "v", "do"))
+        o, lse = att.forward(ql, kl, vl, x["kc"], x["vc"], q_gain=x["qg"], k_gain=x["kg"])
+        dq, dk, dv, dkc, dvc = att.backward(ql, kl, vl, x["kc"], x["vc"], o, lse, dol, q_gain=x["qg"],
+                                            k_gain=x["kg"])
+        np.savez(os.path.join(out_dir, f"r{rank}.npz"), tokens=att.local.tokens, o=o.numpy(), lse=lse.numpy(),
+                 dq=dq.numpy(), dk=dk.numpy(), dv=dv.numpy(),
+                 dkc=np.zeros(0) if dkc is None else dkc.numpy(), dvc=np.zeros(0) if dvc is None else dvc.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+@pytest.mark.parametrize("name,world", [("b45_replica", 2), ("packed_replica", 3), ("kvrange_replica", 2),
+                                        ("tiny", 3), ("small_cached", 2), ("small_cached", 3)])
+def test_gloo_ranks_match_the_single_process_oracle(name, world, tmp_path):
+    import torch.multiprocessing as mp
+    mp.start_processes(_rank_main, args=(world, _free_port(), name, str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    w = _workload(name)
+    x = _inputs(w)
+    ro, rl = oracle.forward(x["q"], x["k"], x["v"], x["kc"], x["vc"], w.videos_array(), w.slices_array(), w.hq,
+                            w.hkv, base=w.rope_base, eps=w.eps, q_gain=x["qg"], k_gain=x["kg"])
+    rq, rk, rv, rkc, rvc, _, _ = oracle.backward(x["q"], x["k"], x["v"], x["kc"], x["vc"], x["do"],
+                                                 w.videos_array(), w.slices_array(), w.hq, w.hkv, base=w.rope_base,
+                                                 eps=w.eps, q_gain=x["qg"], k_gain=x["kg"])
+    seen = np.zeros(w.nq, bool)
+    for r in range(world):
+        z = np.load(os.path.join(tmp_path, f"r{r}.npz"))
+        t = z["tokens"]
+        seen[t] = True
+        np.testing.assert_allclose(z["o"], ro[t], atol=1e-10)
+        fin = np.isfinite(rl[t])
+        assert np.array_equal(np.isfinite(z["lse"]), fin)
+        np.testing.assert_allclose(z["lse"][fin], rl[t][fin], atol=1e-10)
+        np.testing.assert_allclose(z["dq"], rq[t], atol=1e-10)
+        np.testing.assert_allclose(z["dk"], rk[t], atol=1e-10)
+        np.testing.assert_allclose(z["dv"], rv[t], atol=1e-10)
+        if w.num_cache_keys:
+            np.testing.assert_allclose(z["dkc"], rkc, atol=1e-10)
+            np.testing.assert_allclose(z["dvc"], rvc, atol=1e-10)
+    assert seen.all()
+    if name == "small_cached":
+        assert np.abs(rkc).max() > 1e-3          # the cache-gradient path carried something
+
+
+# --------------------------------------------------------------------------- CUDA pieces
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", ["b45_replica", "p720_replica"])
+def test_k_prologue_passes_match_the_oracle(name):
+    from block_causal_attention_b200 import Plan
+    w = W.WORKLOADS[name]
+    p = Plan.from_workload(w)
+    k = W.make_input(w, W.T_K, "cuda")
+    g = torch.Generator().manual_seed(3)
+    kg = (0.5 + torch.rand(w.d, generator=g)).float()
+    dkh = torch.randn((w.nq, w.hkv, w.d), generator=g).float()
+    kh = p.k_prologue(k, kg.cuda())
+    base = torch.randn((w.nq, w.hkv, w.d), generator=g).float()
+    dk = p.k_prologue_bwd(k, dkh.cuda(), kg.cuda(), dk=base.clone().cuda(), accumulate=True)
+    torch.cuda.synchronize()
+    pos = oracle.positions(w.videos_array())
+    ref = oracle.prologue(k.cpu(), pos, w.rope_base, w.eps, kg.double().numpy())
+    assert np.abs(kh.double().cpu().numpy() - ref).max() <= 2 ** -8 * np.abs(ref).max()   # bf16 rounding
+    refd = oracle.prologue_bwd(k.cpu(), pos, dkh.double().numpy(), w.rope_base, w.eps, kg.double().numpy())
+    assert np.abs(dk.double().cpu().numpy() - (refd + base.double().numpy())).max() <= 1e-4
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", ["packed_replica", "kvrange_replica"])
+def test_cuda_engine_one_rank_equals_plain_plan(name):
+    """With one rank the context-parallel path (own keys through k_prologue, needed cache
+    rows gathered, local slices) must give the plain plan's results."""
+    from block_causal_attention_b200 import Plan
+    w = W.WORKLOADS[name]
+    x = W.make_inputs(w, "cuda", with_grad=True)
+    att = CP.ContextParallelAttention(None, 0, 1, w.hq, w.hkv, w.d, w.videos_array(), w.num_cache_keys,
+                                      w.slices_array(), w.rope_base, w.eps, w.o_fp32)
+    o, lse = att.forward(x["q"], x["k"], x["v"], x["k_cache"], x["v_cache"])
+    dq, dk, dv, dkc, dvc = att.backward(x["q"], x["k"], x["v"], x["k_cache"], x["v_cache"], o, lse, x["do"])
+    p = Plan.from_workload(w)
+    o2, l2 = p.fwd(x["q"], x["k"], x["v"], x["k_cache"], x["v_cache"])
+    g2 = p.bwd(x["q"], x["k"], x["v"], x["k_cache"], x["v_cache"], o2, l2, x["do"])
+    torch.cuda.synchronize()
+    assert (o.float() - o2.float()).abs().max().item() <= 1e-2
+    assert (lse - l2).abs().max().item() <= 1e-3
+    for a, b in zip((dq, dk, dv), g2[:3]):
+        assert (a - b).abs().max().item() <= 1e-2
+    if w.num_cache_keys:
+        assert (dkc - g2[3]).abs().max().item() <= 1e-2 and (dvc - g2[4]).abs().max().item() <= 1e-2
