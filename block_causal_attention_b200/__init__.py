@@ -127,11 +127,12 @@ class Plan:
 
     def bwd(self, q, k, v, k_cache, v_cache, o, lse, dout, *, dq=None, dk=None, dv=None, dk_cache=None,
             dv_cache=None, workspace=None, q_gain=None, k_gain=None, stream=None, want_cache_grads=True,
-            param_grads=False):
+            param_grads=False, accumulate=False):
         """Gradients (fp32) w.r.t. q, k, v (new tokens, through QK-Norm + RoPE) and the
         cache; o, lse are the forward's outputs, dout the upstream gradient of O.
         Returns (dq, dk, dv, dk_cache, dv_cache), and with param_grads=True also
-        (dq_gain [D], dk_gain [D], drope_base [3]) appended."""
+        (dq_gain [D], dk_gain [D], drope_base [3]) appended.  accumulate=True adds the five
+        gradients into the given (required) arrays."""
         import torch
         if self.host_only:
             raise BcaError(_abi.BCA_ERR_HOST_ONLY_PLAN, "bwd")
@@ -140,6 +141,9 @@ class Plan:
             raise ValueError("dout: expected contiguous bf16 [Nq, Hq, D]")
         dev = q.device
         f32 = torch.float32
+        if accumulate and (dq is None or dk is None or dv is None or
+                           (self.num_cache_keys and want_cache_grads and (dk_cache is None or dv_cache is None))):
+            raise ValueError("accumulate=True needs the gradient arrays to add into")
         dq = torch.empty((self.nq, self.hq, self.d), device=dev, dtype=f32) if dq is None else dq
         dk = torch.empty((self.nq, self.hkv, self.d), device=dev, dtype=f32) if dk is None else dk
         dv = torch.empty((self.nq, self.hkv, self.d), device=dev, dtype=f32) if dv is None else dv
@@ -149,21 +153,35 @@ class Plan:
             dv_cache = torch.empty(shp, device=dev, dtype=f32) if dv_cache is None else dv_cache
         if workspace is None:
             workspace = self.alloc_workspace(_abi.BCA_PASS_BWD)
-        if not param_grads:
+        if not param_grads and not accumulate:
             rc = self._lib.bca_bwd(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(q_gain),
                                    _ptr(k_gain), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                                    _ptr(dk_cache), _ptr(dv_cache), _ptr(workspace), self._stream(stream))
             _abi.check(rc, "bca_bwd")
             return dq, dk, dv, dk_cache, dv_cache
-        dgq = torch.empty(self.d, device=dev, dtype=f32)
-        dgk = torch.empty(self.d, device=dev, dtype=f32)
-        dbase = torch.empty(3, device=dev, dtype=f32)
+        dgq = torch.empty(self.d, device=dev, dtype=f32) if param_grads else None
+        dgk = torch.empty(self.d, device=dev, dtype=f32) if param_grads else None
+        dbase = torch.empty(3, device=dev, dtype=f32) if param_grads else None
         rc = self._lib.bca_bwd_ex(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(q_gain),
                                   _ptr(k_gain), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                                   _ptr(dk_cache), _ptr(dv_cache), _ptr(dgq), _ptr(dgk), _ptr(dbase),
-                                  _ptr(workspace), self._stream(stream))
+                                  1 if accumulate else 0, _ptr(workspace), self._stream(stream))
         _abi.check(rc, "bca_bwd_ex")
-        return dq, dk, dv, dk_cache, dv_cache, dgq, dgk, dbase
+        out = (dq, dk, dv, dk_cache, dv_cache)
+        return out + (dgq, dgk, dbase) if param_grads else out
+
+    def attn_merge(self, o_a, lse_a, o_b, lse_b, *, o=None, lse=None, stream=None):
+        """O (this plan's O type) and LSE of the whole problem from two partial attentions
+        over disjoint key subsets (fp32 O, LSE [Hq, Nq])."""
+        import torch
+        if o is None:
+            o = torch.empty((self.nq, self.hq, self.d), device=o_a.device,
+                            dtype=torch.float32 if self.o_fp32 else torch.bfloat16)
+        if lse is None:
+            lse = torch.empty((self.hq, self.nq), device=o_a.device, dtype=torch.float32)
+        _abi.check(self._lib.bca_attn_merge(self._h, _ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(o),
+                                            _ptr(lse), self._stream(stream)), "bca_attn_merge")
+        return o, lse
 
     def k_prologue(self, k, k_gain=None, *, out=None, stream=None):
         """Post-prologue keys (bf16 [Nq, Hkv, D]) of the plan's new tokens."""

@@ -35,7 +35,7 @@ BCA_PASS_BWD = 1
 EXPORTS = ("bca_plan_create", "bca_plan_destroy", "bca_plan_get_info", "bca_plan_expand_rows",
            "bca_plan_expand_cols",
            "bca_plan_update_positions", "bca_workspace_bytes", "bca_fwd", "bca_fwd_static_workspace", "bca_bwd",
-           "bca_bwd_ex", "bca_k_prologue", "bca_k_prologue_bwd",
+           "bca_bwd_ex", "bca_attn_merge", "bca_k_prologue", "bca_k_prologue_bwd",
            "bca_profile_enable",
            "bca_profile_read", "bca_status", "bca_error_string")
 BCA_KERNEL_KV_IMAGE = 0
@@ -105,13 +105,15 @@ def lib() -> ctypes.CDLL:
         L.bca_fwd.restype = i32
         L.bca_plan_update_positions.argtypes = [vp, vp, i32, vp]
         L.bca_plan_update_positions.restype = i32
+        L.bca_attn_merge.argtypes = [vp] * 8
+        L.bca_attn_merge.restype = i32
         L.bca_k_prologue.argtypes = [vp] * 5
         L.bca_k_prologue.restype = i32
         L.bca_k_prologue_bwd.argtypes = [vp, vp, vp, vp, vp, i32, vp]
         L.bca_k_prologue_bwd.restype = i32
         L.bca_bwd.argtypes = [vp] * 18
         L.bca_bwd.restype = i32
-        L.bca_bwd_ex.argtypes = [vp] * 21
+        L.bca_bwd_ex.argtypes = [vp] * 19 + [i32, vp, vp]
         L.bca_bwd_ex.restype = i32
         L.bca_fwd_static_workspace.argtypes = [vp] * 11
         L.bca_fwd_static_workspace.restype = i32

@@ -11,7 +11,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libbca.so")
-SOURCES = ["api.cpp", "plan.cpp", "fwd.cu", "fwd_static.cu", "bwd.cu", "prologue_rows.cu"]
+SOURCES = ["api.cpp", "plan.cpp", "fwd.cu", "fwd_static.cu", "bwd.cu", "cp_passes.cu"]
 HEADERS = ["plan.hpp", "kernels.hpp", "sm100.cuh", "prologue.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",

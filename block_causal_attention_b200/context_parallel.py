@@ -117,6 +117,8 @@ class LocalProblem:
     remote_rows: np.ndarray      # global token indices of borrowed keys, sorted
     slices: np.ndarray           # [m, 5] local FULL slices
     area: int
+    slices_held: np.ndarray      # the slices restricted to keys held locally: keys [cache rows | own]
+    slices_borrowed: np.ndarray  # restricted to borrowed keys: keys [borrowed rows | own (unused)]
 
     @property
     def num_cache_keys(self) -> int:
@@ -186,7 +188,18 @@ class ContextParallelPlan:
                     for s0, s1 in zip(starts, ends):
                         out.append((qa, qb, int(seg[s0]), int(seg[s0]) + int(s1 - s0), SLICE_FULL))
         sl = np.asarray(out, np.int64).reshape(-1, 5)
-        return LocalProblem(r, mine, tokens, videos, cache_rows, remote_rows, sl, area)
+        # split at the region boundaries: [0, ncache) cache, [ncache, nc_loc) borrowed, own
+        ncache, nrem = len(cache_rows), len(remote_rows)
+        held, borrowed = [], []
+        for qa, qb, k0, k1, t in out:
+            for lo, hi, dst, shift in ((0, ncache, held, 0), (ncache, nc_loc, borrowed, -ncache),
+                                       (nc_loc, nc_loc + len(tokens), held, -nrem)):
+                a0, a1 = max(k0, lo), min(k1, hi)
+                if a0 < a1:
+                    dst.append((qa, qb, a0 + shift, a1 + shift, t))
+        sh = np.asarray(held, np.int64).reshape(-1, 5)
+        sb = np.asarray(borrowed, np.int64).reshape(-1, 5)
+        return LocalProblem(r, mine, tokens, videos, cache_rows, remote_rows, sl, area, sh, sb)
 
 
 # ----------------------------------------------------------------------------- runtime
@@ -196,9 +209,10 @@ def _default_engine(hq, hkv, d, videos, num_cache_keys, slices, rope_base, eps, 
     return Plan(hq, hkv, d, videos, num_cache_keys, slices, rope_base, eps, o_fp32)
 
 
-def _all_to_all_rows(group, send: List, recv_counts: List[int], row_shape, like):
-    """Rows of `send[dst]` go to rank dst; returns the received rows per source rank.
-    Rows are moved bit-exactly (as 16-bit integers for 16-bit types)."""
+def _all_to_all_rows(group, send: List, recv_counts: List[int], row_shape, like, async_op: bool = False):
+    """Rows of `send[dst]` go to rank dst; returns the received rows per source rank (and,
+    with async_op, the pending work to wait on before reading them).  Rows are moved
+    bit-exactly (as 16-bit integers for 16-bit types)."""
     import torch
     import torch.distributed as dist
     world = len(send)
@@ -209,16 +223,18 @@ def _all_to_all_rows(group, send: List, recv_counts: List[int], row_shape, like)
     as_int = sbuf.dtype in (torch.bfloat16, torch.float16)
     sview = sbuf.view(torch.int16) if as_int else sbuf
     rview = rbuf.view(torch.int16) if as_int else rbuf
+    work = None
     if world == 1:
         rview.copy_(sview)
     else:
-        dist.all_to_all_single(rview, sview, output_split_sizes=list(recv_counts),
-                               input_split_sizes=[int(f.shape[0]) for f in flat], group=group)
+        work = dist.all_to_all_single(rview, sview, output_split_sizes=list(recv_counts),
+                                      input_split_sizes=[int(f.shape[0]) for f in flat], group=group,
+                                      async_op=async_op)
     out, o = [], 0
     for c in recv_counts:
         out.append(rbuf[o:o + c].reshape((c,) + tuple(row_shape)))
         o += c
-    return out
+    return (out, work) if async_op else out
 
 
 class ContextParallelAttention:
@@ -228,19 +244,31 @@ class ContextParallelAttention:
 
     def __init__(self, group, rank: int, world: int, hq: int, hkv: int, d: int, videos, num_cache_keys: int,
                  slices, rope_base=(1e4, 1e4, 1e4), eps: float = 1e-6, o_fp32: bool = False,
-                 engine: Optional[Callable] = None):
+                 engine: Optional[Callable] = None, overlap: bool = False):
+        """overlap=True: attend to the keys held locally while the borrowed ones are in
+        flight, then to the borrowed ones, and merge the two partial results by their
+        log-sum-exps (plans with fp32 O for the parts); the backward runs the borrowed part
+        first so that its gradients travel while the held part computes."""
         self.group, self.rank, self.world = group, int(rank), int(world)
         self.hq, self.hkv, self.d = hq, hkv, d
         self.cp = ContextParallelPlan(world, videos, num_cache_keys, slices)
         self.local = self.cp.local[self.rank]
         eng = engine or _default_engine
-        self.plan = eng(hq, hkv, d, self.local.videos, self.local.num_cache_keys, self.local.slices, rope_base,
-                        eps, o_fp32)
+        lp = self.local
+        self.plan = eng(hq, hkv, d, lp.videos, lp.num_cache_keys, lp.slices, rope_base, eps, o_fp32)
+        self.overlap = bool(overlap) and len(lp.remote_rows) > 0
+        if self.overlap:
+            self.plan_held = eng(hq, hkv, d, lp.videos, len(lp.cache_rows), lp.slices_held, rope_base, eps, True)
+            self.plan_borrowed = eng(hq, hkv, d, lp.videos, len(lp.remote_rows), lp.slices_borrowed, rope_base, eps,
+                                     True)
         self._saved = None
 
     def _gather_keys(self, khat_local, v_local):
-        """Rows of [K-hat | V] of this rank's tokens that the other ranks need, sent; the
-        borrowed rows received, in the order of local.remote_rows."""
+        return self._gather_keys_finish(self._gather_keys_start(khat_local, v_local))
+
+    def _gather_keys_start(self, khat_local, v_local):
+        """Send the rows of [K-hat | V] of this rank's tokens that the other ranks need;
+        returns a handle for _gather_keys_finish (the receive may still be in flight)."""
         import torch
         cp, r = self.cp, self.rank
         pos_in_local = {int(t): j for j, t in enumerate(self.local.tokens)}
@@ -251,7 +279,15 @@ class ContextParallelAttention:
             idx = torch.as_tensor([pos_in_local[int(t)] for t in rows], dtype=torch.long, device=kv.device)
             send.append(kv.index_select(0, idx))
         recv_counts = [len(cp.send_rows[src][r]) for src in range(self.world)]
-        got = _all_to_all_rows(self.group, send, recv_counts, kv.shape[1:], kv)
+        return _all_to_all_rows(self.group, send, recv_counts, kv.shape[1:], kv, async_op=True), recv_counts, kv
+
+    def _gather_keys_finish(self, handle):
+        """The borrowed rows, in the order of local.remote_rows."""
+        import torch
+        (got, work), recv_counts, kv = handle
+        if work is not None:
+            work.wait()
+        cp, r = self.cp, self.rank
         # reorder to local.remote_rows: each source sent its subset in global order
         rr = self.local.remote_rows
         order = {}
@@ -268,6 +304,55 @@ class ContextParallelAttention:
             rem = kv.new_zeros((0,) + tuple(kv.shape[1:]))
         return rem[:, 0], rem[:, 1]
 
+    def _cache_grads(self, dkc, dvc, ncl, like):
+        """Gradients of the global cache: this rank's rows scattered, summed over ranks."""
+        import torch
+        import torch.distributed as dist
+        if not self.cp.nc:
+            return None, None
+        gk = like.new_zeros((self.cp.nc, self.hkv, self.d))
+        gv = like.new_zeros((self.cp.nc, self.hkv, self.d))
+        if ncl:
+            rows = torch.as_tensor(self.local.cache_rows, dtype=torch.long, device=like.device)
+            gk.index_add_(0, rows, dkc[:ncl])
+            gv.index_add_(0, rows, dvc[:ncl])
+        if self.world > 1:
+            dist.all_reduce(gk, group=self.group)
+            dist.all_reduce(gv, group=self.group)
+        return gk, gv
+
+    def _return_grads_start(self, rem_k, rem_v):
+        """Send the borrowed rows' (dK-hat, dV) back to their owners (in flight on return)."""
+        import torch
+        cp, r = self.cp, self.rank
+        grads = torch.stack([rem_k, rem_v], 1)                             # [n_remote, 2, Hkv, D]
+        rpos = {int(t): j for j, t in enumerate(self.local.remote_rows)}
+        send = []
+        for dst in range(self.world):
+            idx = torch.as_tensor([rpos[int(t)] for t in cp.send_rows[dst][r]], dtype=torch.long,
+                                  device=grads.device)
+            send.append(grads.index_select(0, idx))
+        recv_counts = [len(cp.send_rows[r][src]) for src in range(self.world)]
+        return _all_to_all_rows(self.group, send, recv_counts, grads.shape[1:], grads, async_op=True)
+
+    def _return_grads_finish(self, handle, k_local, dk, dv, k_gain):
+        """Add what the other ranks returned for this rank's keys (dK through the prologue)."""
+        import torch
+        got, work = handle
+        if work is not None:
+            work.wait()
+        cp, r = self.cp, self.rank
+        pos_in_local = {int(t): j for j, t in enumerate(self.local.tokens)}
+        dkh = dk.new_zeros(dk.shape)
+        for src in range(self.world):
+            rows = cp.send_rows[r][src]
+            if len(rows):
+                idx = torch.as_tensor([pos_in_local[int(t)] for t in rows], dtype=torch.long, device=dk.device)
+                dkh.index_add_(0, idx, got[src][:, 0])
+                dv.index_add_(0, idx, got[src][:, 1])
+        dk = self.plan.k_prologue_bwd(k_local, dkh, k_gain, dk=dk, accumulate=True)
+        return dk, dv
+
     def _local_cache(self, k_cache, v_cache, rk, rv):
         import torch
         rows = torch.as_tensor(self.local.cache_rows, dtype=torch.long, device=rk.device)
@@ -276,8 +361,25 @@ class ContextParallelAttention:
             return torch.cat([kc, rk], 0), torch.cat([vc, rv], 0)
         return rk, rv
 
+    def _held_cache(self, k_cache, v_cache):
+        import torch
+        if not len(self.local.cache_rows):
+            return None, None
+        rows = torch.as_tensor(self.local.cache_rows, dtype=torch.long, device=k_cache.device)
+        return k_cache.index_select(0, rows), v_cache.index_select(0, rows)
+
     def forward(self, q_local, k_local, v_local, k_cache=None, v_cache=None, q_gain=None, k_gain=None):
         khat = self.plan.k_prologue(k_local, k_gain)
+        if self.overlap:
+            handle = self._gather_keys_start(khat, v_local)
+            kc_h, vc_h = self._held_cache(k_cache, v_cache)
+            o_h, l_h = self.plan_held.fwd(q_local, k_local, v_local, kc_h, vc_h, q_gain=q_gain, k_gain=k_gain)
+            rk, rv = self._gather_keys_finish(handle)
+            o_b, l_b = self.plan_borrowed.fwd(q_local, k_local, v_local, rk, rv, q_gain=q_gain, k_gain=k_gain)
+            o32, lse = self.plan_held.attn_merge(o_h, l_h, o_b, l_b)
+            o = o32 if self.plan.o_fp32 else self.plan.attn_merge(o_h, l_h, o_b, l_b)[0]
+            self._saved = (kc_h, vc_h, rk, rv, o32)
+            return o, lse
         rk, rv = self._gather_keys(khat, v_local)
         kc, vc = self._local_cache(k_cache, v_cache, rk, rv)
         if self.local.num_cache_keys == 0:
@@ -291,41 +393,31 @@ class ContextParallelAttention:
         (summed over ranks, on every rank; None without a cache)."""
         import torch
         import torch.distributed as dist
+        ncl = len(self.local.cache_rows)
+        if self.overlap:
+            kc_h, vc_h, rk, rv, o32 = self._saved
+            # borrowed part first: its key gradients leave while the held part computes
+            dq, dk, dv, rem_k, rem_v = self.plan_borrowed.bwd(q_local, k_local, v_local, rk, rv, o32, lse, do_local,
+                                                              q_gain=q_gain, k_gain=k_gain)
+            handle = self._return_grads_start(rem_k, rem_v)
+            if ncl:
+                dkc = torch.zeros(kc_h.shape, dtype=dk.dtype, device=dk.device)
+                dvc = torch.zeros(vc_h.shape, dtype=dk.dtype, device=dk.device)
+            else:
+                dkc = dvc = None
+            self.plan_held.bwd(q_local, k_local, v_local, kc_h, vc_h, o32, lse, do_local, dq=dq, dk=dk, dv=dv,
+                               dk_cache=dkc, dv_cache=dvc, q_gain=q_gain, k_gain=k_gain, accumulate=True)
+            gk, gv = self._cache_grads(dkc, dvc, ncl, dk)
+            dk, dv = self._return_grads_finish(handle, k_local, dk, dv, k_gain)
+            return dq, dk, dv, gk, gv
         kc, vc = self._saved
         dq, dk, dv, dkc, dvc = self.plan.bwd(q_local, k_local, v_local, kc, vc, o, lse, do_local,
                                              q_gain=q_gain, k_gain=k_gain)
-        ncl = len(self.local.cache_rows)
-        gk = gv = None
-        if self.cp.nc:
-            gk = dk.new_zeros((self.cp.nc, self.hkv, self.d))
-            gv = dk.new_zeros((self.cp.nc, self.hkv, self.d))
-            if ncl:
-                rows = torch.as_tensor(self.local.cache_rows, dtype=torch.long, device=dk.device)
-                gk.index_add_(0, rows, dkc[:ncl])
-                gv.index_add_(0, rows, dvc[:ncl])
-            if self.world > 1:
-                dist.all_reduce(gk, group=self.group)
-                dist.all_reduce(gv, group=self.group)
-        # borrowed rows' gradients go back to their owners
-        cp, r = self.cp, self.rank
+        # the same collective order as the overlapped path (ranks may differ in which path
+        # they take): the returning all-to-all first, then the cache all-reduce
         rem_k = dkc[ncl:] if dkc is not None else dk.new_zeros((0, self.hkv, self.d))
         rem_v = dvc[ncl:] if dvc is not None else dv.new_zeros((0, self.hkv, self.d))
-        grads = torch.stack([rem_k, rem_v], 1)                             # [n_remote, 2, Hkv, D]
-        rpos = {int(t): j for j, t in enumerate(self.local.remote_rows)}
-        send = []
-        for dst in range(self.world):
-            idx = torch.as_tensor([rpos[int(t)] for t in cp.send_rows[dst][r]], dtype=torch.long,
-                                  device=grads.device)
-            send.append(grads.index_select(0, idx))
-        recv_counts = [len(cp.send_rows[r][src]) for src in range(self.world)]
-        got = _all_to_all_rows(self.group, send, recv_counts, grads.shape[1:], grads)
-        pos_in_local = {int(t): j for j, t in enumerate(self.local.tokens)}
-        dkh = dk.new_zeros(dk.shape)
-        for src in range(self.world):
-            rows = cp.send_rows[r][src]
-            if len(rows):
-                idx = torch.as_tensor([pos_in_local[int(t)] for t in rows], dtype=torch.long, device=dk.device)
-                dkh.index_add_(0, idx, got[src][:, 0])
-                dv.index_add_(0, idx, got[src][:, 1])
-        dk = self.plan.k_prologue_bwd(k_local, dkh, k_gain, dk=dk, accumulate=True)
+        handle = self._return_grads_start(rem_k, rem_v)
+        gk, gv = self._cache_grads(dkc, dvc, ncl, dk)
+        dk, dv = self._return_grads_finish(handle, k_local, dk, dv, k_gain)
         return dq, dk, dv, gk, gv

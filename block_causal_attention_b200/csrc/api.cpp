@@ -245,7 +245,7 @@ int bca_fwd(bca_plan_t plan, const void *q, const void *k, const void *v, const 
 int bca_bwd_ex(bca_plan_t plan, const void *q, const void *k, const void *v, const void *k_cache,
                const void *v_cache, const float *q_gain, const float *k_gain, const void *o, const float *lse,
                const void *dout, float *dq, float *dk, float *dv, float *dk_cache, float *dv_cache,
-               float *dq_gain, float *dk_gain, float *drope_base, void *workspace, void *stream) {
+               float *dq_gain, float *dk_gain, float *drope_base, int accumulate, void *workspace, void *stream) {
     if (!plan) return BCA_ERR_INVALID_ARGUMENT;
     bca::Plan &P = plan->plan;
     int rc = check_device(P);
@@ -254,8 +254,8 @@ int bca_bwd_ex(bca_plan_t plan, const void *q, const void *k, const void *v, con
     if (P.nq == 0) {
         // no query: every gradient is zero
         const size_t cb = (size_t)P.nc * P.hkv * P.d * sizeof(float);
-        if (dk_cache && cudaMemsetAsync(dk_cache, 0, cb, s) != cudaSuccess) return BCA_ERR_CUDA;
-        if (dv_cache && cudaMemsetAsync(dv_cache, 0, cb, s) != cudaSuccess) return BCA_ERR_CUDA;
+        if (!accumulate && dk_cache && cudaMemsetAsync(dk_cache, 0, cb, s) != cudaSuccess) return BCA_ERR_CUDA;
+        if (!accumulate && dv_cache && cudaMemsetAsync(dv_cache, 0, cb, s) != cudaSuccess) return BCA_ERR_CUDA;
         if (dq_gain && cudaMemsetAsync(dq_gain, 0, P.d * sizeof(float), s) != cudaSuccess) return BCA_ERR_CUDA;
         if (dk_gain && cudaMemsetAsync(dk_gain, 0, P.d * sizeof(float), s) != cudaSuccess) return BCA_ERR_CUDA;
         if (drope_base && cudaMemsetAsync(drope_base, 0, 3 * sizeof(float), s) != cudaSuccess) return BCA_ERR_CUDA;
@@ -271,7 +271,7 @@ int bca_bwd_ex(bca_plan_t plan, const void *q, const void *k, const void *v, con
     for (const void *p : pptrs)
         if (p && !aligned4(p)) return BCA_ERR_MISALIGNED;
     bca::BwdIO io{q,  k,  v,  k_cache,  v_cache,  q_gain,    k_gain,  o,       lse,       dout,      dq,
-                  dk, dv, dk_cache, dv_cache, workspace, dq_gain, dk_gain, drope_base};
+                  dk, dv, dk_cache, dv_cache, workspace, dq_gain, dk_gain, drope_base, accumulate != 0};
     return bca::launch_bwd(P, io, s);
 }
 
@@ -280,7 +280,22 @@ int bca_bwd(bca_plan_t plan, const void *q, const void *k, const void *v, const 
             const void *dout, float *dq, float *dk, float *dv, float *dk_cache, float *dv_cache,
             void *workspace, void *stream) {
     return bca_bwd_ex(plan, q, k, v, k_cache, v_cache, q_gain, k_gain, o, lse, dout, dq, dk, dv, dk_cache, dv_cache,
-                      nullptr, nullptr, nullptr, workspace, stream);
+                      nullptr, nullptr, nullptr, 0, workspace, stream);
+}
+
+int bca_attn_merge(bca_plan_t plan, const float *o_a, const float *lse_a, const float *o_b, const float *lse_b,
+                   void *o, float *lse, void *stream) {
+    if (!plan) return BCA_ERR_INVALID_ARGUMENT;
+    bca::Plan &P = plan->plan;
+    int rc = check_device(P);
+    if (rc != BCA_OK) return rc;
+    if (P.nq == 0) return BCA_OK;
+    if (!o_a || !lse_a || !o_b || !lse_b || !o || !lse) return BCA_ERR_INVALID_ARGUMENT;
+    const void *ptrs[] = {o_a, o_b, o};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return BCA_ERR_MISALIGNED;
+    if (!aligned4(lse_a) || !aligned4(lse_b) || !aligned4(lse)) return BCA_ERR_MISALIGNED;
+    return bca::launch_attn_merge(P, o_a, lse_a, o_b, lse_b, o, lse, static_cast<cudaStream_t>(stream));
 }
 
 int bca_k_prologue(bca_plan_t plan, const void *k, const float *k_gain, void *k_hat, void *stream) {

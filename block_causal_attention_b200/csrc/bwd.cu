@@ -105,6 +105,7 @@ struct BwdArgs {
     float *dgain_k, *dbase;  // optional parameter gradients (K gain; RoPE bases, shared with Q)
     float coef[24];          // d(base_a^(-k/P))/d(base_a) at [8 a + k]
     int32_t tbase;           // absolute frame of packed t = 0
+    int accumulate;          // add dK, dV (and the cache's) into the outputs instead of writing them
     int *status;
 };
 
@@ -123,6 +124,7 @@ struct DqArgs {
     float *dgain_q, *dbase;  // optional parameter gradients (Q gain; RoPE bases, shared with K)
     float coef[24];
     int32_t tbase;
+    int accumulate;  // add dQ into the output instead of writing it
 };
 
 // Power-of-two scale sc applied to dS before its fp16 rounding: 1 unless the bound
@@ -141,6 +143,19 @@ __device__ __forceinline__ float ds_scale(const float *bounds) {
 // atomic max of non-negative floats through their (order-preserving) bit patterns
 __device__ __forceinline__ void atomic_max_nonneg(float *addr, float v) {
     atomicMax(reinterpret_cast<int *>(addr), __float_as_int(v));
+}
+
+// Write (or, when accumulating, add) four fp32 values.
+__device__ __forceinline__ void store_or_add4(float *p, float4 v, int accumulate) {
+    float4 *q = reinterpret_cast<float4 *>(p);
+    if (accumulate) {
+        const float4 o = *q;
+        v.x += o.x;
+        v.y += o.y;
+        v.z += o.z;
+        v.w += o.w;
+    }
+    *q = v;
 }
 
 // core-matrix image offset (in 16-byte chunks) of chunk c (8 columns) of row r in a
@@ -722,8 +737,10 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                 if (dst) {
 #pragma unroll
                     for (int c = 0; c < D / 4; ++c)
-                        reinterpret_cast<float4 *>(dst)[c] = make_float4(acc[4 * c] * inv_sc, acc[4 * c + 1] * inv_sc,
-                                                                         acc[4 * c + 2] * inv_sc, acc[4 * c + 3] * inv_sc);
+                        store_or_add4(dst + 4 * c,
+                                      make_float4(acc[4 * c] * inv_sc, acc[4 * c + 1] * inv_sc, acc[4 * c + 2] * inv_sc,
+                                                  acc[4 * c + 3] * inv_sc),
+                                      a.accumulate);
                 }
             } else {
                 float gk[D];
@@ -745,7 +762,8 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                 if (dst) {
 #pragma unroll
                     for (int c = 0; c < D / 4; ++c)
-                        reinterpret_cast<float4 *>(dst)[c] = make_float4(gk[4 * c], gk[4 * c + 1], gk[4 * c + 2], gk[4 * c + 3]);
+                        store_or_add4(dst + 4 * c, make_float4(gk[4 * c], gk[4 * c + 1], gk[4 * c + 2], gk[4 * c + 3]),
+                                      a.accumulate);
                 }
             }
         }
@@ -801,9 +819,10 @@ __global__ void __launch_bounds__(128) bwd_dq_kernel(DqArgs a) {
             qk_param_grads<D>(x, g, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps, a.coef,
                               a.tbase, pg, pb);
         qk_prologue_bwd<D>(x, g, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps);
-        float4 *dst = reinterpret_cast<float4 *>(a.dq + row * D);
+        float *dst = a.dq + row * D;
 #pragma unroll
-        for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(g[4 * c], g[4 * c + 1], g[4 * c + 2], g[4 * c + 3]);
+        for (int c = 0; c < D / 4; ++c)
+            store_or_add4(dst + 4 * c, make_float4(g[4 * c], g[4 * c + 1], g[4 * c + 2], g[4 * c + 3]), a.accumulate);
     }
     if (want_pg) {
         // the block's 128 rows: warp sums, then one add per value for the block
@@ -958,6 +977,7 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     ba.dbase = io.drope_base;
     for (int i = 0; i < 24; ++i) ba.coef[i] = P.rope_base_coef[i];
     ba.tbase = P.rope_tbase;
+    ba.accumulate = io.accumulate;
     ba.status = P.d_status;
     {
         ProfScope ps(P, BCA_KERNEL_BWD, stream);
@@ -985,6 +1005,7 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     da.dbase = io.drope_base;
     for (int i = 0; i < 24; ++i) da.coef[i] = P.rope_base_coef[i];
     da.tbase = P.rope_tbase;
+    da.accumulate = io.accumulate;
     {
         ProfScope ps(P, BCA_KERNEL_BWD_DQ, stream);
         if (P.nq > 0) bwd_dq_kernel<D><<<dim3((unsigned)P.nqt, (unsigned)P.hq), 128, 0, stream>>>(da);

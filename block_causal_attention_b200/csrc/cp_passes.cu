@@ -1,5 +1,7 @@
-// The key prologue (QK-Norm + 3D RoPE) and its backward over the rows of a plan's new
-// tokens, as stand-alone passes.  The attention kernels fuse these steps; the passes
+// Passes for context parallelism.  (1) The key prologue (QK-Norm + 3D RoPE) and its
+// backward over the rows of a plan's new tokens, as stand-alone passes.  (2) The merge of
+// two partial attentions over disjoint key subsets by their log-sum-exps, so that a rank
+// can attend to the keys it holds while the borrowed ones are still in flight.  The attention kernels fuse these steps; the passes
 // exist for context-parallel use, where a key row's post-prologue value K-hat is computed
 // once by the rank that owns the token and sent to the ranks that attend to it, and the
 // gradients those ranks return for K-hat are mapped back through the prologue by the
@@ -113,7 +115,78 @@ int dispatch_rows(const Plan &P, const RowArgs &a, bool backward, cudaStream_t s
     }
 }
 
+struct MergeArgs {
+    const float *o_a, *lse_a, *o_b, *lse_b;
+    void *o;
+    float *lse;
+    int o_fp32;
+    int64_t nq;
+    int hq;
+};
+
+// one thread per (query, head): with m = max(lse_a, lse_b), w = exp(lse - m):
+// O = (w_a O_a + w_b O_b) / (w_a + w_b), LSE = m + log(w_a + w_b); no visible key in
+// either part gives O = 0, LSE = -inf
+template <int D>
+__global__ void __launch_bounds__(128) attn_merge_kernel(MergeArgs a) {
+    const int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int h = blockIdx.y;
+    if (q >= a.nq) return;
+    const size_t row = (size_t)q * a.hq + h;
+    const size_t li = (size_t)h * a.nq + q;
+    const float la = a.lse_a[li], lb = a.lse_b[li];
+    const float m = fmaxf(la, lb);
+    float wa = 0.f, wb = 0.f, lse = -INFINITY;
+    if (m > -INFINITY) {
+        wa = la > -INFINITY ? __expf(la - m) : 0.f;
+        wb = lb > -INFINITY ? __expf(lb - m) : 0.f;
+        const float s = wa + wb;
+        lse = m + __logf(s);
+        wa /= s;
+        wb /= s;
+    }
+    float o[D];
+    const float4 *pa = reinterpret_cast<const float4 *>(a.o_a + row * D);
+    const float4 *pb = reinterpret_cast<const float4 *>(a.o_b + row * D);
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c) {
+        const float4 x = pa[c], y = pb[c];
+        o[4 * c] = wa * x.x + wb * y.x;
+        o[4 * c + 1] = wa * x.y + wb * y.y;
+        o[4 * c + 2] = wa * x.z + wb * y.z;
+        o[4 * c + 3] = wa * x.w + wb * y.w;
+    }
+    if (a.o_fp32) {
+        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.o) + row * D);
+#pragma unroll
+        for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+    } else {
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.o) + row * D);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) dst[c] = pack_chunk_bf16<D>(o, c);
+    }
+    a.lse[li] = lse;
+}
+
+template <int D>
+int launch_merge(const MergeArgs &a, cudaStream_t stream) {
+    attn_merge_kernel<D><<<dim3((unsigned)((a.nq + 127) / 128), (unsigned)a.hq), 128, 0, stream>>>(a);
+    return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
+}
+
 }  // namespace
+
+int launch_attn_merge(const Plan &P, const float *o_a, const float *lse_a, const float *o_b, const float *lse_b,
+                      void *o, float *lse, cudaStream_t stream) {
+    if (P.nq == 0) return BCA_OK;
+    MergeArgs a{o_a, lse_a, o_b, lse_b, o, lse, (P.flags & BCA_O_FP32) ? 1 : 0, P.nq, P.hq};
+    switch (P.d) {
+        case 24: return launch_merge<24>(a, stream);
+        case 32: return launch_merge<32>(a, stream);
+        case 48: return launch_merge<48>(a, stream);
+        default: return BCA_ERR_UNSUPPORTED;
+    }
+}
 
 int launch_k_prologue(const Plan &P, const void *k, const float *k_gain, void *k_hat, cudaStream_t stream) {
     RowArgs a = row_args(P, k, k_gain);

@@ -27,6 +27,7 @@ struct BwdIO {
     float *dq, *dk, *dv, *dk_cache, *dv_cache;
     void *workspace;
     float *dq_gain, *dk_gain, *drope_base;  // optional parameter gradients (NULL = not wanted)
+    int accumulate;                         // add dq, dk, dv, dk_cache, dv_cache into the outputs
 };
 
 // Bytes of each K-hat / V image (all KV heads, all k-tiles), 256-byte rounded.
@@ -42,6 +43,9 @@ size_t bwd_workspace_bytes(const Plan &plan);
 
 // K prologue over the plan's new tokens (bf16 K-hat rows) and its backward
 // (dk = or += J^T dk_hat), for context-parallel exchange of post-prologue keys.
+// O and LSE of one problem from the O (fp32) and LSE of two disjoint key subsets.
+int launch_attn_merge(const Plan &plan, const float *o_a, const float *lse_a, const float *o_b, const float *lse_b,
+                      void *o, float *lse, cudaStream_t stream);
 int launch_k_prologue(const Plan &plan, const void *k, const float *k_gain, void *k_hat, cudaStream_t stream);
 int launch_k_prologue_bwd(const Plan &plan, const void *k, const float *k_gain, const float *dk_hat, float *dk,
                           int accumulate, cudaStream_t stream);

@@ -212,12 +212,28 @@ int bca_bwd(bca_plan_t plan, const void *q, const void *k, const void *v,
  *   drope_base : fp32 [3], dL/d(rope_base[t, h, w]), summed over Q and new K rows.
  * Any of the three may be NULL (not computed); non-NULL ones are overwritten (4-byte
  * aligned).  The sums are formed with atomic adds, so their last bits may differ between
- * runs.  Everything else is as bca_bwd, which is this call with the three set to NULL. */
+ * runs.  accumulate != 0 adds dq, dk, dv, dk_cache and dv_cache into the given arrays
+ * instead of overwriting them (the three parameter gradients are still overwritten): the
+ * gradients of a problem whose keys are split over several plans are the sums of the
+ * plans' gradients, each plan given the O and LSE of the whole problem.  Everything else
+ * is as bca_bwd, which is this call with the three pointers NULL and accumulate = 0. */
 int bca_bwd_ex(bca_plan_t plan, const void *q, const void *k, const void *v,
                const void *k_cache, const void *v_cache, const float *q_gain,
                const float *k_gain, const void *o, const float *lse, const void *dout,
                float *dq, float *dk, float *dv, float *dk_cache, float *dv_cache,
-               float *dq_gain, float *dk_gain, float *drope_base, void *workspace, void *stream);
+               float *dq_gain, float *dk_gain, float *drope_base, int accumulate, void *workspace,
+               void *stream);
+
+/* O and LSE of one problem from two partial attentions over disjoint key subsets (the
+ * Flex-Flash-Attention merge of partial results by their log-sum-exps: MAGI-1 research
+ * notes, "Infra > MagiAttention"), so that context parallelism can attend to the keys a
+ * rank holds while the borrowed ones are in flight.  o_a, o_b: fp32 [Nq][Hq][D] (plans
+ * with BCA_O_FP32); lse_a, lse_b, lse: fp32 [Hq][Nq] (natural log, -inf = no key);
+ * o: [Nq][Hq][D] in this plan's O type.  With m = max(lse_a, lse_b) and w = exp(lse - m):
+ * O = (w_a O_a + w_b O_b) / (w_a + w_b), LSE = m + log(w_a + w_b); rows with no key in
+ * either part get O = 0, LSE = -inf.  Sizes from the plan (Nq, Hq, D). */
+int bca_attn_merge(bca_plan_t plan, const float *o_a, const float *lse_a, const float *o_b,
+                   const float *lse_b, void *o, float *lse, void *stream);
 
 /* The key prologue of bca_fwd (QK-Norm + 3D RoPE at the plan's positions of its new
  * tokens) as a stand-alone pass, and its backward.  Used by context parallelism: the

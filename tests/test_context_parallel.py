@@ -60,10 +60,14 @@ def test_causal_slices_are_rejected():
 # --------------------------------------------------------------------------- gloo ranks
 
 class OracleEngine:
-    """The attention engine on the fp64 oracle (test infrastructure only)."""
+    """The attention engine on the fp64 oracle (test infrastructure only).  Its backward
+    takes the O and LSE of the whole problem, as the CUDA plan's does, so that a plan over
+    a subset of the keys yields that subset's share of the gradients."""
+
+    o_fp32 = True
 
     def __init__(self, hq, hkv, d, videos, nc, slices, base, eps, o_fp32):
-        self.hq, self.hkv, self.d = hq, hkv, d
+        self.hq, self.hkv, self.d, self.nc = hq, hkv, d, nc
         self.videos, self.slices, self.base, self.eps = np.asarray(videos), np.asarray(slices), base, eps
         self.pos = oracle.positions(self.videos) if len(self.videos) else np.zeros((0, 3), np.int32)
 
@@ -79,12 +83,54 @@ class OracleEngine:
                                 eps=self.eps, q_gain=q_gain, k_gain=k_gain)
         return torch.from_numpy(o), torch.from_numpy(lse)
 
-    def bwd(self, q, k, v, kc, vc, o, lse, do, q_gain=None, k_gain=None):
-        dq, dk, dv, dkc, dvc, _, _ = oracle.backward(q, k, v, kc, vc, do, self.videos, self.slices, self.hq,
-                                                     self.hkv, base=self.base, eps=self.eps, q_gain=q_gain,
-                                                     k_gain=k_gain)
-        t = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a))
-        return t(dq), t(dk), t(dv), t(dkc), t(dvc)
+    def attn_merge(self, o_a, lse_a, o_b, lse_b):
+        la, lb = lse_a.numpy(), lse_b.numpy()
+        m = np.maximum(la, lb)
+        fin = np.isfinite(m)
+        ms = np.where(fin, m, 0.0)
+        wa = np.where(np.isfinite(la), np.exp(la - ms), 0.0)
+        wb = np.where(np.isfinite(lb), np.exp(lb - ms), 0.0)
+        tot = wa + wb
+        lse = np.where(fin, ms + np.log(np.where(fin, tot, 1.0)), -np.inf)
+        sa, sb = np.where(fin, wa / np.where(fin, tot, 1.0), 0.0), np.where(fin, wb / np.where(fin, tot, 1.0), 0.0)
+        o = o_a.numpy() * sa[..., None] + o_b.numpy() * sb[..., None]
+        return torch.from_numpy(o), torch.from_numpy(lse)
+
+    def bwd(self, q, k, v, kc, vc, o, lse, do, q_gain=None, k_gain=None, dq=None, dk=None, dv=None,
+            dk_cache=None, dv_cache=None, accumulate=False):
+        nq, nc = q.shape[0], self.nc
+        qh = oracle.prologue(q, self.pos, self.base, self.eps, q_gain)
+        kh = oracle.prologue(k, self.pos, self.base, self.eps, k_gain)
+        if nc:
+            kh = np.concatenate([np.asarray(kc, np.float64), kh])
+            vv = np.concatenate([np.asarray(vc, np.float64), np.asarray(v, np.float64)])
+        else:
+            vv = np.asarray(v, np.float64)
+        M = oracle.mask_dense(self.slices, nq, nc + nq).astype(bool)
+        O, L, dO = np.asarray(o, np.float64), np.asarray(lse, np.float64), np.asarray(do, np.float64)
+        G = self.hq // self.hkv
+        dqh, dkh, dvv = np.zeros_like(qh), np.zeros_like(kh), np.zeros_like(vv)
+        sc = 1.0 / np.sqrt(self.d)
+        for h in range(self.hq):
+            g = h // G
+            S = qh[:, h] @ kh[:, g].T * sc
+            Lh = L[:, h][:, None]
+            P = np.where(M & np.isfinite(Lh), np.exp(S - np.where(np.isfinite(Lh), Lh, 0.0)), 0.0)
+            dP = dO[:, h] @ vv[:, g].T
+            dS = P * (dP - (dO[:, h] * O[:, h]).sum(-1)[:, None])
+            dqh[:, h] = dS @ kh[:, g] * sc
+            dkh[:, g] += dS.T @ qh[:, h] * sc
+            dvv[:, g] += P.T @ dO[:, h]
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a))
+        gq = t(oracle.prologue_bwd(q, self.pos, dqh, self.base, self.eps, q_gain))
+        gk = t(oracle.prologue_bwd(k, self.pos, dkh[nc:], self.base, self.eps, k_gain))
+        out = [gq, gk, t(dvv[nc:]), t(dkh[:nc]) if nc else None, t(dvv[:nc]) if nc else None]
+        if accumulate:
+            for dst, add in zip((dq, dk, dv, dk_cache, dv_cache), out):
+                if dst is not None:
+                    dst += add
+            return dq, dk, dv, dk_cache, dv_cache
+        return tuple(out)
 
 
 def _small_cached():
@@ -113,7 +159,7 @@ def _inputs(w):
     return x
 
 
-def _rank_main(rank, world, port, name, out_dir):
+def _rank_main(rank, world, port, name, out_dir, overlap=False):
     import torch.distributed as dist
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
@@ -122,7 +168,8 @@ def _rank_main(rank, world, port, name, out_dir):
         w = _workload(name)
         x = _inputs(w)
         att = CP.ContextParallelAttention(None, rank, world, w.hq, w.hkv, w.d, w.videos_array(), w.num_cache_keys,
-                                          w.slices_array(), w.rope_base, w.eps, engine=OracleEngine)
+                                          w.slices_array(), w.rope_base, w.eps, engine=OracleEngine,
+                                          overlap=overlap)
         tok = torch.as_tensor(att.local.tokens, dtype=torch.long)
         ql, kl, vl, dol = (x[n].index_select(0, tok) for n in ("q", "k", "v", "do"))
         o, lse = att.forward(ql, kl, vl, x["kc"], x["vc"], q_gain=x["qg"], k_gain=x["kg"])
@@ -143,12 +190,15 @@ def _free_port():
     return p
 
 
-@pytest.mark.parametrize("name,world", [("b45_replica", 2), ("packed_replica", 3), ("kvrange_replica", 2),
-                                        ("tiny", 3), ("small_cached", 2), ("small_cached", 3)])
-def test_gloo_ranks_match_the_single_process_oracle(name, world, tmp_path):
+@pytest.mark.parametrize("name,world,overlap", [("b45_replica", 2, False), ("packed_replica", 3, False),
+                                                ("kvrange_replica", 2, True), ("tiny", 3, True),
+                                                ("small_cached", 2, False), ("small_cached", 3, True)])
+def test_gloo_ranks_match_the_single_process_oracle(name, world, overlap, tmp_path):
+    """overlap=True: each rank attends to the keys it holds while the borrowed ones are in
+    flight and merges the two partial results by their log-sum-exps."""
     import torch.multiprocessing as mp
-    mp.start_processes(_rank_main, args=(world, _free_port(), name, str(tmp_path)), nprocs=world, join=True,
-                       start_method="spawn")
+    mp.start_processes(_rank_main, args=(world, _free_port(), name, str(tmp_path), overlap), nprocs=world,
+                       join=True, start_method="spawn")
     w = _workload(name)
     x = _inputs(w)
     ro, rl = oracle.forward(x["q"], x["k"], x["v"], x["kc"], x["vc"], w.videos_array(), w.slices_array(), w.hq,
@@ -221,3 +271,55 @@ def test_cuda_engine_one_rank_equals_plain_plan(name):
         assert (a - b).abs().max().item() <= 1e-2
     if w.num_cache_keys:
         assert (dkc - g2[3]).abs().max().item() <= 1e-2 and (dvc - g2[4]).abs().max().item() <= 1e-2
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", ["p720_replica", "packed_replica"])
+def test_cuda_split_by_key_location_equals_unsplit(name):
+    """Rank 0 of a 2-rank split, on one GPU: the plans over held and borrowed keys, merged
+    by their log-sum-exps (bca_attn_merge), and their backwards added into the same arrays
+    (accumulate), give the unsplit local plan's O, LSE and gradients."""
+    from block_causal_attention_b200 import Plan
+    w = W.WORKLOADS[name]
+    x = W.make_inputs(w, "cuda", with_grad=True)
+    lp = CP.ContextParallelPlan(2, w.videos_array(), w.num_cache_keys, w.slices_array()).local[0]
+    assert len(lp.remote_rows) > 0
+    mk = lambda nc, sl, f32: Plan(w.hq, w.hkv, w.d, lp.videos, nc, sl, w.rope_base, w.eps, f32)
+    full = mk(lp.num_cache_keys, lp.slices, True)
+    held = mk(len(lp.cache_rows), lp.slices_held, True)
+    bor = mk(len(lp.remote_rows), lp.slices_borrowed, True)
+    dev = "cuda"
+    tok = torch.as_tensor(lp.tokens, device=dev)
+    ql, kl, vl, dol = (x[n].index_select(0, tok) for n in ("q", "k", "v", "do"))
+    khat_all = Plan.from_workload(w).k_prologue(x["k"])
+    rr = torch.as_tensor(lp.remote_rows, device=dev)
+    rk, rv = khat_all.index_select(0, rr), x["v"].index_select(0, rr)
+    if len(lp.cache_rows):
+        cr = torch.as_tensor(lp.cache_rows, device=dev)
+        kch, vch = x["k_cache"].index_select(0, cr), x["v_cache"].index_select(0, cr)
+        kcf, vcf = torch.cat([kch, rk]), torch.cat([vch, rv])
+    else:
+        kch = vch = None
+        kcf, vcf = rk, rv
+    of, lf = full.fwd(ql, kl, vl, kcf, vcf)
+    oh, lh = held.fwd(ql, kl, vl, kch, vch)
+    ob, lb = bor.fwd(ql, kl, vl, rk, rv)
+    om, lm = held.attn_merge(oh, lh, ob, lb)
+    gf = full.bwd(ql, kl, vl, kcf, vcf, of, lf, dol)
+    dq, dk, dv, rem_k, rem_v = bor.bwd(ql, kl, vl, rk, rv, om, lm, dol)
+    dkc = torch.zeros(kch.shape, dtype=torch.float32, device=dev) if kch is not None else None
+    dvc = torch.zeros(vch.shape, dtype=torch.float32, device=dev) if vch is not None else None
+    held.bwd(ql, kl, vl, kch, vch, om, lm, dol, dq=dq, dk=dk, dv=dv, dk_cache=dkc, dv_cache=dvc, accumulate=True)
+    torch.cuda.synchronize()
+    for p in (full, held, bor):
+        assert p.status() == 0
+    fin = torch.isfinite(lf)
+    assert torch.equal(fin, torch.isfinite(lm))
+    assert (lm[fin] - lf[fin]).abs().max().item() <= 1e-3
+    assert (om - of).abs().max().item() <= 1e-2
+    for a, b in ((dq, gf[0]), (dk, gf[1]), (dv, gf[2])):
+        assert (a - b).abs().max().item() <= 1e-2
+    ncl = len(lp.cache_rows)
+    assert (rem_k - gf[3][ncl:]).abs().max().item() <= 1e-2 and (rem_v - gf[4][ncl:]).abs().max().item() <= 1e-2
+    if ncl:
+        assert (dkc - gf[3][:ncl]).abs().max().item() <= 1e-2 and (dvc - gf[4][:ncl]).abs().max().item() <= 1e-2
