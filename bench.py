@@ -45,10 +45,15 @@ def _args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "fwdbwd"], default="fwdbwd")
+    ap.add_argument("--fp8", action="store_true",
+                    help="forward with e4m3 tensor-core operands (BCA_FWD_FP8_E4M3; needs --pass fwd)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=8, help="query rows (all heads) in the oracle sample")
-    return ap.parse_args()
+    a = ap.parse_args()
+    if a.fp8 and a.pass_ != "fwd":
+        ap.error("--fp8 is a forward-only variant: use it with --pass fwd")
+    return a
 
 
 def _peaks():
@@ -209,7 +214,7 @@ def run_ours(a):
 
     t0 = time.perf_counter()
     plan = Plan(hq, hkv, w.d, w.videos_array(), w.num_cache_keys, w.slices_array(), w.rope_base, w.eps,
-                w.o_fp32)
+                w.o_fp32, fp8=a.fp8)
     plan_ms = 1e3 * (time.perf_counter() - t0)
     info = plan.info()
 
@@ -389,6 +394,10 @@ def run_ours(a):
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_kind = f"bf16 dense, sustained, {peak_src}"
+    if a.fp8:   # e4m3 contraction: the measured bf16 peak x the nominal fp8 / bf16 ratio (4.5 / 2.25)
+        peak_sus, peak_burst = 2.0 * peak_sus, 2.0 * peak_burst
+        peak_kind = f"e4m3 dense = 2 x bf16 dense sustained ({peak_src}; nominal fp8/bf16 ratio)"
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.txt")
     if os.path.exists(tpath):
@@ -399,7 +408,7 @@ def run_ours(a):
                     traffic = float(parts[2])
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
                 "frac": achieved / peak_sus, "traffic": traffic,
-                "kernel": dom, "peak_kind": f"bf16 dense, sustained, {peak_src}",
+                "kernel": dom, "peak_kind": peak_kind,
                 "frac_of_burst_peak": achieved / peak_burst,
                 "kernel_share_of_step": (ms_bwd if dom == "bwd_kernel" else ms_fwd) / max(1e-9, ms_all)}
     fwd_tflops = flops_fwd_launch / (avg_fwd_ms * 1e-3) / 1e12
@@ -416,8 +425,8 @@ def run_ours(a):
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": elapsed_ms / a.steps, "higher_is_better": True,
-            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "pass": a.pass_, "nq": w.nq, "nk": w.nk, "hq": w.hq, "hkv": w.hkv,
+            "scaling": "strong", "vs_baseline": None, "dtype": "e4m3" if a.fp8 else "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "pass": a.pass_, "operands": "e4m3" if a.fp8 else "bf16/fp16", "nq": w.nq, "nk": w.nk, "hq": w.hq, "hkv": w.hkv,
                        "d": w.d, "visible_pairs_per_head": pairs,
                        "parallelism": f"head-parallel x{world}" if world > 1 else "1 GPU",
                        "l2": "inputs larger than L2 (Q 1.06 GB, K/V images 0.4 GB, O 1.06 GB)",

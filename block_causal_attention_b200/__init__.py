@@ -26,9 +26,10 @@ class Plan:
 
     def __init__(self, hq: int, hkv: int, d: int, videos, num_cache_keys: int = 0, slices=None,
                  rope_base=(1e4, 1e4, 1e4), eps: float = 1e-6, o_fp32: bool = False,
-                 host_only: bool = False, test_force_timeout: bool = False):
+                 host_only: bool = False, test_force_timeout: bool = False, fp8: bool = False):
+        """fp8=True: forward with e4m3 tensor-core operands (BCA_FWD_FP8_E4M3; forward only)."""
         flags = (_abi.BCA_O_FP32 if o_fp32 else 0) | (_abi.BCA_PLAN_HOST_ONLY if host_only else 0) | \
-            (_abi.BCA_TEST_FORCE_TIMEOUT if test_force_timeout else 0)
+            (_abi.BCA_TEST_FORCE_TIMEOUT if test_force_timeout else 0) | (_abi.BCA_FWD_FP8_E4M3 if fp8 else 0)
         prob, keep = _abi.make_problem(hq, hkv, d, videos, num_cache_keys, slices, rope_base, eps, flags)
         self._lib = _abi.lib()
         self._h = _abi.ctypes.c_void_p()
@@ -37,6 +38,7 @@ class Plan:
         _abi.check(rc, "bca_plan_create")
         self.hq, self.hkv, self.d = int(hq), int(hkv), int(d)
         self.o_fp32 = bool(o_fp32)
+        self.fp8 = bool(fp8)
         self.host_only = bool(host_only)
         self.num_cache_keys = int(num_cache_keys)
         inf = self.info()
@@ -47,9 +49,9 @@ class Plan:
             self.device_index = torch.cuda.current_device()
 
     @classmethod
-    def from_workload(cls, w, host_only: bool = False, o_fp32: Optional[bool] = None) -> "Plan":
+    def from_workload(cls, w, host_only: bool = False, o_fp32: Optional[bool] = None, fp8: bool = False) -> "Plan":
         return cls(w.hq, w.hkv, w.d, w.videos_array(), w.num_cache_keys, w.slices_array(),
-                   w.rope_base, w.eps, w.o_fp32 if o_fp32 is None else o_fp32, host_only)
+                   w.rope_base, w.eps, w.o_fp32 if o_fp32 is None else o_fp32, host_only, fp8=fp8)
 
     def update_positions(self, videos, stream=None) -> None:
         """Move the videos' start frames (t0) of this plan, same geometry otherwise: only the

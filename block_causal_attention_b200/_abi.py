@@ -28,6 +28,7 @@ BCA_SLICE_CAUSAL = 1
 BCA_O_FP32 = 0x1
 BCA_PLAN_HOST_ONLY = 0x2
 BCA_TEST_FORCE_TIMEOUT = 0x4
+BCA_FWD_FP8_E4M3 = 0x8
 BCA_PASS_FWD = 0
 BCA_PASS_BWD = 1
 

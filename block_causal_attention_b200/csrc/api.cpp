@@ -248,6 +248,7 @@ int bca_bwd_ex(bca_plan_t plan, const void *q, const void *k, const void *v, con
                float *dq_gain, float *dk_gain, float *drope_base, int accumulate, void *workspace, void *stream) {
     if (!plan) return BCA_ERR_INVALID_ARGUMENT;
     bca::Plan &P = plan->plan;
+    if (P.flags & BCA_FWD_FP8_E4M3) return BCA_ERR_UNSUPPORTED;  // the e4m3 path is forward only
     int rc = check_device(P);
     if (rc != BCA_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -47,6 +47,9 @@ struct KVArgs {
     float eps;
     __half *kimg;
     __nv_bfloat16 *vimg;
+    // e4m3 images (plans with BCA_FWD_FP8_E4M3)
+    uint8_t *kimg8, *vimg8;
+    float *vamax;  // [hkv] max |V| over the new and the cache rows
 };
 
 struct FwdArgs {
@@ -57,6 +60,8 @@ struct FwdArgs {
     int32_t axis_off0, axis_off1, axis_off2;
     const __half *kimg;
     const __nv_bfloat16 *vimg;
+    const uint8_t *kimg8, *vimg8;  // e4m3 images (FP8 kernel only)
+    const float *vamax;            // [hkv] max |V|, for the power-of-two V scale (FP8 only)
     const Item *items;
     const int32_t *run_off;
     const Run *runs;
@@ -137,20 +142,118 @@ __global__ void __launch_bounds__(128) kv_image_kernel(KVArgs a) {
     }
 }
 
+// ------------------------------------------------------------------ e4m3 images
+//
+// The FP8 forward (plans created with BCA_FWD_FP8_E4M3) feeds the tensor cores e4m3
+// operands: K-hat as it is (RMS-normalised, so |x| <= sqrt(D) * max|gain| stays far
+// inside e4m3's +-448), and V divided by a power of two 2^e per KV head, chosen from the
+// largest |V| so that V / 2^e <= 448; the epilogue multiplies O by 2^e again (exact).
+
+// Exponent e of the power-of-two V scale: amax / 448 in [2^(e-1), 2^e), so V / 2^e < 448
+// (0 for amax == 0).  Exact, from amax's own binary exponent: amax = m * 2^f with m in
+// [0.5, 1) and 448 = 0.875 * 2^9, so e = f - 8 when m >= 0.875, else f - 9.
+__device__ __forceinline__ int v8_scale_exp(float amax) {
+    if (!(amax > 0.f)) return 0;
+    int f;
+    const float m = frexpf(amax, &f);
+    return m >= 0.875f ? f - 8 : f - 9;
+}
+
+// amax[g] = max |V| over the new rows and the cache rows of KV head g (amax zeroed before).
+template <int D>
+__global__ void __launch_bounds__(256) v_amax_kernel(KVArgs a) {
+    const int64_t row = (int64_t)blockIdx.x * 256 + threadIdx.x;  // key row in [0, nk)
+    const int g = blockIdx.y;
+    float m = 0.f;
+    if (row < a.nk) {
+        float x[D];
+        if (row < a.nc) load_row_bf16<D>(a.vc + ((size_t)row * a.hkv + g) * D, x);
+        else load_row_bf16<D>(a.v + ((size_t)(row - a.nc) * a.hkv + g) * D, x);
+#pragma unroll
+        for (int d = 0; d < D; ++d) m = fmaxf(m, fabsf(x[d]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    // non-negative floats order like their bit patterns
+    if ((threadIdx.x & 31) == 0 && m > 0.f) atomicMax(reinterpret_cast<int *>(a.vamax + g), __float_as_int(m));
+}
+
+// e4m3 tile images, one (k-tile, KV head) per block:
+//   K-hat: 128 keys x DP8, K-major; core (d chunk c of 16, key group kg of 8) at
+//          (c * 16 + kg) * 128 bytes, element (key, d) at + (key % 8) * 16 + d % 16.
+//   V^T  : DPAD x 128 keys, K-major; core (key chunk kc of 16, d group dg of 8) at
+//          (kc * DPAD/8 + dg) * 128 bytes, element (d, key) at + (d % 8) * 16 + key % 16.
+template <int D>
+__global__ void __launch_bounds__(128) kv_image8_kernel(KVArgs a) {
+    constexpr int DPAD = Geo<D>::DPAD;
+    constexpr int DP8 = Geo<D>::DP8;
+    __shared__ float sv[128][DPAD + 1];
+    const int t = threadIdx.x;
+    const int64_t kt = blockIdx.x;
+    const int g = blockIdx.y;
+    const int64_t key = kt * 128 + t;
+    const size_t tile = (size_t)g * a.nkt + kt;
+
+    float x[D];
+    if (key < a.nc) {
+        load_row_bf16<D>(a.kc + ((size_t)key * a.hkv + g) * D, x);
+    } else if (key < a.nk) {
+        const int64_t n = key - a.nc;
+        load_row_bf16<D>(a.k + ((size_t)n * a.hkv + g) * D, x);
+        qk_prologue<D>(x, __ldg(a.pos + n), a.k_gain, a.rope, a.axis_off0, a.axis_off1, a.axis_off2, a.eps,
+                       1.0f);
+    } else {
+#pragma unroll
+        for (int d = 0; d < D; ++d) x[d] = 0.f;
+    }
+    uint4 *kout = reinterpret_cast<uint4 *>(a.kimg8 + tile * Geo<D>::K8_TILE_BYTES);
+#pragma unroll
+    for (int c = 0; c < DP8 / 16; ++c) kout[(c * 16 + t / 8) * 8 + (t % 8)] = pack_chunk_e4m3<D>(x, c);
+
+    const float mul = ldexpf(1.0f, -v8_scale_exp(a.vamax[g]));
+    if (key < a.nc) {
+        load_row_bf16<D>(a.vc + ((size_t)key * a.hkv + g) * D, x);
+    } else if (key < a.nk) {
+        load_row_bf16<D>(a.v + ((size_t)(key - a.nc) * a.hkv + g) * D, x);
+    } else {
+#pragma unroll
+        for (int d = 0; d < D; ++d) x[d] = 0.f;
+    }
+#pragma unroll
+    for (int d = 0; d < DPAD; ++d) sv[t][d] = d < D ? x[d] * mul : 0.f;
+    __syncthreads();
+    uint4 *vout = reinterpret_cast<uint4 *>(a.vimg8 + tile * Geo<D>::V8_TILE_BYTES);
+#pragma unroll
+    for (int i = 0; i < DPAD / 16; ++i) {
+        const int c = t + 128 * i;  // 16-byte row index = (kc * DPAD/8 + dg) * 8 + dd
+        const int dd = c % 8, dg = (c / 8) % (DPAD / 8), kc = c / DPAD;
+        const int d = dg * 8 + dd;
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            w[e] = pack_e4m3x4(sv[kc * 16 + 4 * e][d], sv[kc * 16 + 4 * e + 1][d], sv[kc * 16 + 4 * e + 2][d],
+                               sv[kc * 16 + 4 * e + 3][d]);
+        vout[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 // ------------------------------------------------------------------ attention kernel
 
-template <int D>
+// F8: e4m3 Q-hat, K-hat, P and V^T (k-granule 32), else fp16 Q-hat / K-hat and bf16 P / V.
+template <int D, bool F8>
 struct FwdSmem {
     static constexpr int DPAD = Geo<D>::DPAD;
+    static constexpr int DP8 = Geo<D>::DP8;
     static constexpr int STAGES = 4;
-    static constexpr int Q_BYTES = 128 * DPAD * 2;
-    static constexpr int P_BYTES = 128 * 128 * 2;
-    static constexpr int TILE = Geo<D>::TILE_BYTES;
+    static constexpr int Q_BYTES = F8 ? 128 * DP8 : 128 * DPAD * 2;
+    static constexpr int P_BYTES = F8 ? 128 * 128 : 128 * 128 * 2;
+    static constexpr int KTILE = F8 ? Geo<D>::K8_TILE_BYTES : Geo<D>::TILE_BYTES;
+    static constexpr int VTILE = F8 ? Geo<D>::V8_TILE_BYTES : Geo<D>::TILE_BYTES;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_P = OFF_Q + 2 * Q_BYTES;
     static constexpr int OFF_K = OFF_P + 2 * P_BYTES;
-    static constexpr int OFF_V = OFF_K + STAGES * TILE;
-    static constexpr int OFF_BAR = OFF_V + STAGES * TILE;
+    static constexpr int OFF_V = OFF_K + STAGES * KTILE;
+    static constexpr int OFF_BAR = OFF_V + STAGES * VTILE;
     // barriers
     static constexpr int B_KV_FULL = 0;
     static constexpr int B_KV_EMPTY = STAGES;
@@ -205,13 +308,13 @@ __device__ __forceinline__ bool warp_wait_or_abort(uint32_t bar, uint32_t parity
     return __all_sync(0xffffffffu, ok);
 }
 
-template <int D>
+template <int D, bool F8>
 __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
-    using L = FwdSmem<D>;
+    using L = FwdSmem<D, F8>;
     constexpr int DPAD = L::DPAD;
     constexpr int STAGES = L::STAGES;
-    constexpr uint32_t IDESC_S = idesc_f32acc(128, 128, kFmtF16);
-    constexpr uint32_t IDESC_PV = idesc_f32acc(128, DPAD, kFmtBF16);
+    constexpr uint32_t IDESC_S = idesc_f32acc(128, 128, F8 ? kFmtE4M3 : kFmtF16);
+    constexpr uint32_t IDESC_PV = idesc_f32acc(128, DPAD, F8 ? kFmtE4M3 : kFmtBF16);
 
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
@@ -267,10 +370,14 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
                 if (j >= STAGES &&
                     !wait_or_abort(bar(L::B_KV_EMPTY + stage), ((j / STAGES) - 1) & 1, a.status, abort_flag, a.timeout_ns))
                     break;
-                const size_t tile = ((size_t)g * a.nkt + cur.kt) * (128 * DPAD);
-                mbar_arrive_expect_tx(bar(L::B_KV_FULL + stage), 2 * L::TILE);
-                bulk_g2s(sbase + L::OFF_K + stage * L::TILE, a.kimg + tile, L::TILE, bar(L::B_KV_FULL + stage));
-                bulk_g2s(sbase + L::OFF_V + stage * L::TILE, a.vimg + tile, L::TILE, bar(L::B_KV_FULL + stage));
+                const size_t tile = (size_t)g * a.nkt + cur.kt;
+                const void *ksrc = F8 ? (const void *)(a.kimg8 + tile * L::KTILE)
+                                      : (const void *)(a.kimg + tile * (128 * DPAD));
+                const void *vsrc = F8 ? (const void *)(a.vimg8 + tile * L::VTILE)
+                                      : (const void *)(a.vimg + tile * (128 * DPAD));
+                mbar_arrive_expect_tx(bar(L::B_KV_FULL + stage), L::KTILE + L::VTILE);
+                bulk_g2s(sbase + L::OFF_K + stage * L::KTILE, ksrc, L::KTILE, bar(L::B_KV_FULL + stage));
+                bulk_g2s(sbase + L::OFF_V + stage * L::VTILE, vsrc, L::VTILE, bar(L::B_KV_FULL + stage));
                 ++issued;
             }
             // every issued copy must have landed before the CTA may exit
@@ -286,25 +393,32 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
                       wait_or_abort(bar(L::B_Q_READY + 1), 0, a.status, abort_flag, a.timeout_ns) &&
                       wait_or_abort(bar(L::B_KV_FULL + 0), 0, a.status, abort_flag, a.timeout_ns);
             tc_fence_after();
+            // Both operands K-major with no swizzle: a core matrix is 8 rows x 16 bytes (8
+            // fp16/bf16 or 16 e4m3 elements), core matrices adjacent in K lie 2048 bytes
+            // apart (V: (DPAD/8) * 128), adjacent in M/N 128 bytes apart.  One MMA consumes
+            // two core matrices of K (16 elements at 16 bits, 32 at 8 bits).
             auto issue_s = [&](int slot, int stage) {
                 const uint32_t qa = sbase + L::OFF_Q + slot * L::Q_BYTES;
-                const uint32_t kb = sbase + L::OFF_K + stage * L::TILE;
+                const uint32_t kb = sbase + L::OFF_K + stage * L::KTILE;
+                constexpr int KSTEPS = F8 ? L::DP8 / 32 : DPAD / 16;
 #pragma unroll
-                for (int kk = 0; kk < DPAD / 16; ++kk) {
+                for (int kk = 0; kk < KSTEPS; ++kk) {
                     const uint64_t ad = smem_desc(qa + kk * 4096, 2048, 128);
                     const uint64_t bd = smem_desc(kb + kk * 4096, 2048, 128);
-                    mma_f16(tbase + L::COL_S + 128 * slot, ad, bd, IDESC_S, kk > 0);
+                    if constexpr (F8) mma_f8(tbase + L::COL_S + 128 * slot, ad, bd, IDESC_S, kk > 0);
+                    else mma_f16(tbase + L::COL_S + 128 * slot, ad, bd, IDESC_S, kk > 0);
                 }
             };
             auto issue_pv = [&](int slot, int stage, bool acc) {
                 const uint32_t pa = sbase + L::OFF_P + slot * L::P_BYTES;
-                const uint32_t vb = sbase + L::OFF_V + stage * L::TILE;
+                const uint32_t vb = sbase + L::OFF_V + stage * L::VTILE;
                 constexpr uint32_t VLBO = (DPAD / 8) * 128;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
+                for (int kk = 0; kk < (F8 ? 4 : 8); ++kk) {
                     const uint64_t ad = smem_desc(pa + kk * 4096, 2048, 128);
                     const uint64_t bd = smem_desc(vb + kk * 2 * VLBO, VLBO, 128);
-                    mma_f16(tbase + L::COL_O + 64 * slot, ad, bd, IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+                    if constexpr (F8) mma_f8(tbase + L::COL_O + 64 * slot, ad, bd, IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+                    else mma_f16(tbase + L::COL_O + 64 * slot, ad, bd, IDESC_PV, (acc || kk > 0) ? 1u : 0u);
                 }
             };
             if (ok) {
@@ -352,19 +466,26 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
         const bool live = qrow < a.nq;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
 
-        {   // Q prologue into shared memory (fp16, core-matrix layout, K-major A operand)
+        {   // Q prologue into shared memory (core-matrix layout, K-major A operand): fp16 with
+            // the softmax scale folded in, or e4m3 unscaled (the scale is applied to S in fp32,
+            // keeping the normalised values in e4m3's normal range)
             float x[D];
             if (live) {
                 load_row_bf16<D>(a.q + ((size_t)qrow * a.hq + h) * D, x);
                 qk_prologue<D>(x, __ldg(a.pos + qrow), a.q_gain, a.rope, a.axis_off0, a.axis_off1, a.axis_off2,
-                               a.eps, a.qscale);
+                               a.eps, F8 ? 1.0f : a.qscale);
             } else {
 #pragma unroll
                 for (int d = 0; d < D; ++d) x[d] = 0.f;
             }
             uint4 *qs = reinterpret_cast<uint4 *>(smem + L::OFF_Q + slot * L::Q_BYTES);
+            if constexpr (F8) {
 #pragma unroll
-            for (int c = 0; c < DPAD / 8; ++c) qs[(c * 16 + row / 8) * 8 + row % 8] = pack_chunk_f16<D>(x, c);
+                for (int c = 0; c < L::DP8 / 16; ++c) qs[(c * 16 + row / 8) * 8 + row % 8] = pack_chunk_e4m3<D>(x, c);
+            } else {
+#pragma unroll
+                for (int c = 0; c < DPAD / 8; ++c) qs[(c * 16 + row / 8) * 8 + row % 8] = pack_chunk_f16<D>(x, c);
+            }
             fence_proxy_async_smem();
             mbar_arrive(bar(L::B_Q_READY + slot));
         }
@@ -401,6 +522,7 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
             float mx = s[0];
 #pragma unroll
             for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+            if constexpr (F8) mx *= a.qscale;  // S in log2 units (the scale is positive)
             float alpha = 1.f;
             bool rescale = false;
             if (mx > m_ref + 8.0f) {  // lazy rescaling: move the reference only when it grows by > 2^8
@@ -412,7 +534,7 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
             float sum = 0.f;
 #pragma unroll
             for (int c = 0; c < 128; ++c) {
-                s[c] = ex2(s[c] - msub);
+                s[c] = F8 ? ex2(fmaf(s[c], a.qscale, -msub)) : ex2(s[c] - msub);
                 sum += s[c];
             }
             l = l * alpha + sum;
@@ -435,12 +557,24 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
                     tmem_wait_st();
                 }
             }
-            // P (bf16) in the core-matrix layout of the K-major A operand
+            // P (bf16, or e4m3: P <= 2^8 under the lazy rescale, inside e4m3's range) in the
+            // core-matrix layout of the K-major A operand
+            if constexpr (F8) {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const uint4 u = make_uint4(pack_bf16x2(s[8 * c + 0], s[8 * c + 1]), pack_bf16x2(s[8 * c + 2], s[8 * c + 3]),
-                                           pack_bf16x2(s[8 * c + 4], s[8 * c + 5]), pack_bf16x2(s[8 * c + 6], s[8 * c + 7]));
-                ps[(c * 16 + row / 8) * 8 + row % 8] = u;
+                for (int c = 0; c < 8; ++c) {
+                    const float *v = s + 16 * c;
+                    ps[(c * 16 + row / 8) * 8 + row % 8] =
+                        make_uint4(pack_e4m3x4(v[0], v[1], v[2], v[3]), pack_e4m3x4(v[4], v[5], v[6], v[7]),
+                                   pack_e4m3x4(v[8], v[9], v[10], v[11]), pack_e4m3x4(v[12], v[13], v[14], v[15]));
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const uint4 u =
+                        make_uint4(pack_bf16x2(s[8 * c + 0], s[8 * c + 1]), pack_bf16x2(s[8 * c + 2], s[8 * c + 3]),
+                                   pack_bf16x2(s[8 * c + 4], s[8 * c + 5]), pack_bf16x2(s[8 * c + 6], s[8 * c + 7]));
+                    ps[(c * 16 + row / 8) * 8 + row % 8] = u;
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -467,7 +601,8 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
         }
         if (live) {
             const bool any = l > 0.f;
-            const float inv = any ? 1.0f / l : 0.f;
+            float inv = any ? 1.0f / l : 0.f;
+            if constexpr (F8) inv = ldexpf(inv, v8_scale_exp(a.vamax[g]));  // undo V / 2^e
             if (a.o_fp32) {
                 float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.o) + ((size_t)qrow * a.hq + h) * D);
 #pragma unroll
@@ -497,10 +632,15 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
 
 template <int D>
 int launch_fwd_d(Plan &P, const FwdIO &io, cudaStream_t stream) {
-    using L = FwdSmem<D>;
+    const bool f8 = (P.flags & BCA_FWD_FP8_E4M3) != 0;
     const size_t img = kv_image_bytes(P);
     auto *kimg = static_cast<__half *>(io.workspace);
     auto *vimg = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(io.workspace) + img);
+    // e4m3 images share the workspace: K-hat at 0, V^T after it, the V amax after both
+    uint8_t *ws8 = static_cast<uint8_t *>(io.workspace);
+    const size_t k8 = ((size_t)P.hkv * (size_t)P.nkt * Geo<D>::K8_TILE_BYTES + 255) / 256 * 256;
+    const size_t v8 = ((size_t)P.hkv * (size_t)P.nkt * Geo<D>::V8_TILE_BYTES + 255) / 256 * 256;
+    float *vamax = reinterpret_cast<float *>(ws8 + k8 + v8);
 
     KVArgs ka;
     ka.k = static_cast<const __nv_bfloat16 *>(io.k);
@@ -520,7 +660,16 @@ int launch_fwd_d(Plan &P, const FwdIO &io, cudaStream_t stream) {
     ka.eps = P.eps;
     ka.kimg = kimg;
     ka.vimg = vimg;
-    {
+    ka.kimg8 = ws8;
+    ka.vimg8 = ws8 + k8;
+    ka.vamax = vamax;
+    if (f8) {
+        if (cudaMemsetAsync(vamax, 0, (size_t)P.hkv * sizeof(float), stream) != cudaSuccess) return BCA_ERR_CUDA;
+        ProfScope ps(P, BCA_KERNEL_KV_IMAGE, stream);
+        if (P.nk > 0)
+            v_amax_kernel<D><<<dim3((unsigned)((P.nk + 255) / 256), (unsigned)P.hkv), 256, 0, stream>>>(ka);
+        kv_image8_kernel<D><<<dim3((unsigned)P.nkt, (unsigned)P.hkv), 128, 0, stream>>>(ka);
+    } else {
         ProfScope ps(P, BCA_KERNEL_KV_IMAGE, stream);
         kv_image_kernel<D><<<dim3((unsigned)P.nkt, (unsigned)P.hkv), 128, 0, stream>>>(ka);
     }
@@ -536,6 +685,9 @@ int launch_fwd_d(Plan &P, const FwdIO &io, cudaStream_t stream) {
     fa.axis_off2 = P.rope_axis_off[2];
     fa.kimg = kimg;
     fa.vimg = vimg;
+    fa.kimg8 = ws8;
+    fa.vimg8 = ws8 + k8;
+    fa.vamax = vamax;
     fa.items = P.d_items;
     fa.run_off = P.d_run_off;
     fa.runs = P.d_runs;
@@ -554,7 +706,8 @@ int launch_fwd_d(Plan &P, const FwdIO &io, cudaStream_t stream) {
     fa.skip_loads = (P.flags & BCA_TEST_FORCE_TIMEOUT) ? 1 : 0;
     {
         ProfScope ps(P, BCA_KERNEL_FWD, stream);
-        fwd_kernel<D><<<(unsigned)P.items.size(), 384, L::BYTES, stream>>>(fa);
+        if (f8) fwd_kernel<D, true><<<(unsigned)P.items.size(), 384, FwdSmem<D, true>::BYTES, stream>>>(fa);
+        else fwd_kernel<D, false><<<(unsigned)P.items.size(), 384, FwdSmem<D, false>::BYTES, stream>>>(fa);
     }
     if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
     return BCA_OK;
@@ -567,7 +720,9 @@ size_t kv_image_bytes(const Plan &P) {
     return (b + 255) / 256 * 256;
 }
 
-size_t fwd_workspace_bytes(const Plan &P) { return 2 * kv_image_bytes(P); }
+// The bf16 K-hat and V images, or (FP8 plans) the smaller e4m3 images plus 256 bytes for
+// the per-KV-head V amax.
+size_t fwd_workspace_bytes(const Plan &P) { return 2 * kv_image_bytes(P) + ((size_t)P.hkv * 4 + 255) / 256 * 256; }
 
 // The attention kernel needs more than 48 KB of dynamic shared memory; the attribute
 // is set once per plan (at creation, on the plan's device) so that no launch path makes
@@ -577,10 +732,20 @@ int prepare_fwd(const Plan &P) {
         return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
     };
     bool ok = true;
+    const bool f8 = (P.flags & BCA_FWD_FP8_E4M3) != 0;
     switch (P.d) {
-        case 24: ok = set((const void *)fwd_kernel<24>, FwdSmem<24>::BYTES); break;
-        case 32: ok = set((const void *)fwd_kernel<32>, FwdSmem<32>::BYTES); break;
-        case 48: ok = set((const void *)fwd_kernel<48>, FwdSmem<48>::BYTES); break;
+        case 24:
+            ok = f8 ? set((const void *)fwd_kernel<24, true>, FwdSmem<24, true>::BYTES)
+                    : set((const void *)fwd_kernel<24, false>, FwdSmem<24, false>::BYTES);
+            break;
+        case 32:
+            ok = f8 ? set((const void *)fwd_kernel<32, true>, FwdSmem<32, true>::BYTES)
+                    : set((const void *)fwd_kernel<32, false>, FwdSmem<32, false>::BYTES);
+            break;
+        case 48:
+            ok = f8 ? set((const void *)fwd_kernel<48, true>, FwdSmem<48, true>::BYTES)
+                    : set((const void *)fwd_kernel<48, false>, FwdSmem<48, false>::BYTES);
+            break;
         default: return BCA_ERR_UNSUPPORTED;
     }
     return ok ? BCA_OK : BCA_ERR_CUDA;

@@ -121,7 +121,8 @@ void compile_q_tile(const Plan &P, int64_t qt, TileOut &out) {
 
 int validate_problem(const bca_problem *p, Plan &P) {
     if (!p) return BCA_ERR_INVALID_ARGUMENT;
-    if (p->flags & ~(BCA_O_FP32 | BCA_PLAN_HOST_ONLY | BCA_TEST_FORCE_TIMEOUT)) return BCA_ERR_INVALID_ARGUMENT;
+    if (p->flags & ~(BCA_O_FP32 | BCA_PLAN_HOST_ONLY | BCA_TEST_FORCE_TIMEOUT | BCA_FWD_FP8_E4M3))
+        return BCA_ERR_INVALID_ARGUMENT;
     if (p->num_q_heads <= 0 || p->num_kv_heads <= 0) return BCA_ERR_INVALID_ARGUMENT;
     if (p->num_q_heads % p->num_kv_heads != 0) return BCA_ERR_UNSUPPORTED;
     if ((p->num_q_heads / p->num_kv_heads) % 2 != 0) return BCA_ERR_UNSUPPORTED;

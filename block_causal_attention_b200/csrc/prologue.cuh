@@ -21,6 +21,10 @@ struct Geo {
     static constexpr int DPAD = (D + 15) / 16 * 16;     // MMA k-granule for bf16 is 16
     static constexpr int PAIRS = (D / 2) / 3;           // RoPE pairs per axis
     static constexpr int TILE_BYTES = 128 * DPAD * 2;   // one K-hat or V tile image
+    // 8-bit operands: the MMA k-granule is 32 elements, a core-matrix row 16 elements
+    static constexpr int DP8 = (D + 31) / 32 * 32;      // head dim of the e4m3 Q-hat / K-hat images
+    static constexpr int K8_TILE_BYTES = 128 * DP8;     // one e4m3 K-hat tile image
+    static constexpr int V8_TILE_BYTES = DPAD * 128;    // one e4m3 V^T tile image
 };
 
 // ------------------------------------------------------------------ prologue math
@@ -80,6 +84,24 @@ __device__ __forceinline__ uint4 pack_chunk_f16(const float (&x)[D], int c) {
         const float lo = d0 < D ? x[d0] : 0.f;
         const float hi = d0 + 1 < D ? x[d0 + 1] : 0.f;
         w[e] = sm100::pack_f16x2(lo, hi);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Pack values [16c, 16c+16) of x (zero past D), each multiplied by mul, into one
+// 16-byte chunk of e4m3.
+template <int D>
+__device__ __forceinline__ uint4 pack_chunk_e4m3(const float (&x)[D], int c, float mul = 1.f) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int d = c * 16 + 4 * e + u;
+            v[u] = d < D ? x[d] * mul : 0.f;
+        }
+        w[e] = sm100::pack_e4m3x4(v[0], v[1], v[2], v[3]);
     }
     return make_uint4(w[0], w[1], w[2], w[3]);
 }

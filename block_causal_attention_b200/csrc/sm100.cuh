@@ -152,6 +152,7 @@ __host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, uint32_t ab_fo
            | ((uint32_t)(M >> 4) << 24);      // M / 16
 }
 constexpr uint32_t kFmtF16 = 0, kFmtBF16 = 1;
+constexpr uint32_t kFmtE4M3 = 0;  // A/B format code of e4m3 under kind::f8f6f4
 
 // Same with an operand's major-ness chosen: a_mn / b_mn = 1 marks that operand
 // MN-major (its 16-byte core-matrix rows run along M resp. N instead of K).
@@ -167,6 +168,18 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T with 8-bit float operands (kind::f8f6f4; both
+// operands e4m3 here), K = 32 elements per instruction, fp32 accumulator.
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
@@ -271,6 +284,19 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Two fp32 values to two e4m3 bytes (round to nearest even, saturating at +-448):
+// lo in the low byte.  The conversion instruction puts its first source in the high byte.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Four fp32 values to four e4m3 bytes, x0 in the lowest byte.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float x0, float x1, float x2, float x3) {
+    return pack_e4m3x2(x0, x1) | (pack_e4m3x2(x2, x3) << 16);
 }
 
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {

@@ -75,6 +75,20 @@ extern "C" {
 #define BCA_TEST_FORCE_TIMEOUT 0x4u /* failure-detection test: bca_fwd's K/V loads are not
                                        issued and its waits give up after 1 ms, so every
                                        CTA records BCA_ERR_DEVICE_TIMEOUT and exits cleanly */
+#define BCA_FWD_FP8_E4M3 0x8u /* forward with e4m3 tensor-core operands (the 8-bit float
+                                 MMAs of sm_100a): Q-hat and K-hat rounded to e4m3, V to
+                                 e4m3 after division by a power of two per KV head (from
+                                 max|V|, undone in the epilogue), P to e4m3; accumulation,
+                                 softmax and LSE stay fp32.  The MAGI-1 pages quantise
+                                 their linear layers to FP8 at inference (Notes,
+                                 inference infrastructure, real-time streaming scenario:
+                                 W8A8 SmoothQuant); this applies the format to attention.
+                                 Error: each score and each P carries a relative rounding
+                                 error of at most 2^-4 (e4m3's 3-bit significand), so
+                                 O is accurate to a few percent of |V| / sqrt(effective
+                                 number of keys), not to bf16 precision.  Forward only:
+                                 bca_bwd / bca_bwd_ex on such a plan return
+                                 BCA_ERR_UNSUPPORTED (train with bf16 plans). */
 
 /* bca_workspace_bytes(pass) */
 #define BCA_PASS_FWD 0
@@ -105,7 +119,8 @@ typedef struct {
                                    every chunk of the first video */
     float rope_base[3];         /* RoPE base per axis (t, h, w) */
     float norm_eps;             /* QK-Norm epsilon */
-    uint32_t flags;             /* BCA_O_FP32 | BCA_PLAN_HOST_ONLY | BCA_TEST_FORCE_TIMEOUT */
+    uint32_t flags;             /* BCA_O_FP32 | BCA_PLAN_HOST_ONLY | BCA_TEST_FORCE_TIMEOUT |
+                                   BCA_FWD_FP8_E4M3 */
 } bca_problem;
 
 typedef struct bca_plan_s *bca_plan_t;

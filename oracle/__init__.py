@@ -300,3 +300,138 @@ def backward_rows(q_rows, rows, k, v, k_cache, v_cache, do_rows, videos, slices,
     qh = prologue(qr, pos[rows], base, eps, q_gain)
     dqh, O, lse = attn_bwd_rows(qh, rows, kh, vv, do_rows, slices, hq, hkv)
     return prologue_bwd(qr, pos[rows], dqh, base, eps, q_gain)
+
+
+# ---------------------------------------------------------------------------
+# e4m3 operands (the FP8 forward variant)
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0          # largest finite e4m3 value: 1.75 * 2^8
+E4M3_MIN_NORMAL = 2.0 ** -6
+E4M3_SUBNORMAL_STEP = 2.0 ** -9
+
+
+def round_e4m3(x) -> np.ndarray:
+    """Round to the nearest e4m3 value (ties to an even significand), saturating at
+    +-448.  The format (OCP 8-bit floating point, E4M3): 1 sign bit, 4 exponent bits
+    with bias 7, 3 significand bits, no infinities; normal values (1 + m/8) * 2^e for
+    e in [-6, 8] (the top code of e = 8 is NaN, so the largest is 1.75 * 2^8), and
+    subnormals m/8 * 2^-6.  In a binade [2^e, 2^(e+1)) the spacing is 2^(e-3); below
+    2^-6 it is 2^-9."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    e = np.floor(np.log2(np.maximum(a, E4M3_MIN_NORMAL)))
+    step = np.where(a < E4M3_MIN_NORMAL, E4M3_SUBNORMAL_STEP, 2.0 ** (e - 3))
+    r = np.rint(a / step) * step                      # rint: halves go to the even multiple
+    r = np.minimum(r, E4M3_MAX)
+    return np.where(np.isnan(x), np.nan, np.copysign(r, x))
+
+
+def e4m3_scale_exponent(amax: float) -> int:
+    """Exponent e of the power-of-two scale that brings V into e4m3's range: the e with
+    amax / 448 in [2^(e-1), 2^e), so V / 2^e < 448 (0 when amax is 0).  Taken from the
+    exact binary exponent of amax: amax = m * 2^f with m in [0.5, 1) and 448 = 0.875 * 2^9,
+    so e = f - 8 when m >= 0.875, else f - 9."""
+    if not amax > 0:
+        return 0
+    m, f = np.frexp(float(amax))
+    return int(f - 8 if m >= 0.875 else f - 9)
+
+
+def _e4m3_step(a):
+    """Spacing of e4m3 values around |x| = a (2^(e-3) in the binade [2^e, 2^(e+1)))."""
+    e = np.floor(np.log2(np.maximum(a, E4M3_MIN_NORMAL)))
+    return np.where(a < E4M3_MIN_NORMAL, E4M3_SUBNORMAL_STEP, 2.0 ** (e - 3))
+
+
+def _e4m3_undecided(x, window=2e-6):
+    """Step of the elements whose e4m3 rounding a computation carrying an error of
+    window * max(|x|, 1) could take either way (within that distance of a rounding
+    midpoint), else 0."""
+    a = np.abs(x)
+    step = _e4m3_step(a)
+    frac = a / step - np.floor(a / step)
+    near = np.abs(frac - 0.5) * step < window * np.maximum(a, 1.0)
+    return np.where(near & (a > 0), step, 0.0)
+
+
+def forward_fp8(q, k, v, k_cache, v_cache, videos, slices, hq, hkv,
+                base=(1e4, 1e4, 1e4), eps=1e-6, q_gain=None, k_gain=None, rows=None, q_rows=None):
+    """The forward with e4m3 operands, and the spread its last rounding leaves.
+
+    Same method as ``forward`` with the tensor-core operands rounded to e4m3: Q-hat and
+    K-hat after the prologue (unscaled; the softmax scale 1/sqrt(D) multiplies the
+    fp64 score), and V divided by 2^e per KV head (``e4m3_scale_exponent`` of max|V|
+    over the new and the cache rows), rounded, and multiplied back.  The scores, the
+    softmax and P V are then exact (fp64).  Cache keys are used as given (post-prologue).
+
+    The GPU kernel also rounds P to e4m3 before P V, at a per-row reference that the
+    online softmax chooses (P <= 2^8), so its P differs from this P by a relative
+    rounding error of at most 2^-4 per element in e4m3's normal range, and by at most
+    2^-10 (half the subnormal step) in the kernel's P units below it, a unit at least
+    exp(lse - max s) in normalised probability.  Treating those errors as independent
+    and uniform gives the standard deviation returned as ``sd``:
+        sd[i,h,d]^2 = sum_j ((2^-4/sqrt 3)^2 p_ij^2 + (2^-10/sqrt 3)^2 exp(2 (max_j s_ij - lse_i)))
+                      * (v_jd - o_id)^2.
+    A Q-hat or K-hat element computed in fp32 (the kernel's prologue) within about 2e-6
+    of an e4m3 rounding midpoint may round to the other neighbour, moving score s_ij by
+    at most that element's step times its partner's magnitude / sqrt(D).  ``flip`` is
+    the p-weighted sum of those possible score moves per (row, head), a first-order bound
+    of the LSE change they can cause (and, times max_j |v_jd - o_id|, of the O change);
+    it is 0 for rows no undecided element reaches.
+    Returns (O [nr,Hq,D], LSE [nr,Hq], sd [nr,Hq,D], flip [nr,Hq], vdev [nr,Hq,D] =
+    max_j |v_jd| over the KV group plus |o_id|, a bound of max_j |v_jd - o_id|)."""
+    pos = positions(videos)
+    if rows is None:
+        rows = np.arange(pos.shape[0], dtype=np.int64)
+    rows = np.asarray(rows, dtype=np.int64)
+    qr = _f64(q_rows) if q_rows is not None else _f64(q)[rows]
+    D = qr.shape[-1]
+    nc = 0 if k_cache is None else int(k_cache.shape[0])
+    kh = full_keys(prologue(k, pos, base, eps, k_gain), k_cache)
+    vv = full_keys(v, v_cache)
+    qh = prologue(qr, pos[rows], base, eps, q_gain)
+    uq = _e4m3_undecided(qh)
+    uk = _e4m3_undecided(kh)
+    uk[:nc] = 0.0                                   # cache keys are bf16 values: rounded exactly alike
+    q8 = round_e4m3(qh)
+    k8 = round_e4m3(kh)
+    v8 = np.empty_like(vv)
+    for g in range(hkv):
+        e = e4m3_scale_exponent(np.abs(vv[:, g, :]).max() if vv.shape[0] else 0.0)
+        v8[:, g, :] = round_e4m3(vv[:, g, :] / 2.0 ** e) * 2.0 ** e
+    nk = kh.shape[0]
+    vis = np.stack([mask_row(slices, nk, int(i)) for i in rows]) if len(rows) else np.zeros((0, nk), bool)
+    G = hq // hkv
+    nr = len(rows)
+    O = np.zeros((nr, hq, D))
+    lse = np.full((nr, hq), -np.inf)
+    sd = np.zeros((nr, hq, D))
+    flip = np.zeros((nr, hq))
+    vdev = np.zeros((nr, hq, D))
+    rel = 2.0 ** -4 / np.sqrt(3.0)
+    absu = 2.0 ** -10 / np.sqrt(3.0)
+    for h in range(hq):
+        g = h // G
+        s = (q8[:, h, :] @ k8[:, g, :].T) / np.sqrt(D)
+        s = np.where(vis, s, -np.inf)
+        smax = s.max(axis=1, initial=-np.inf)
+        live = np.isfinite(smax)
+        sm = np.where(live, smax, 0.0)
+        ex = np.exp(s - sm[:, None])
+        tot = ex.sum(axis=1)
+        l_ = np.where(live, sm + np.log(np.where(live, tot, 1.0)), -np.inf)
+        p = ex / np.where(live, tot, 1.0)[:, None]
+        vg = v8[:, g, :]
+        o = p @ vg
+        # sum_j w_ij (v_jd - o_id)^2 = w@v^2 - 2 o (w@v) + o^2 sum_j w_ij
+        w = (rel * p) ** 2 + (absu * np.where(live, np.exp(sm - l_), 0.0))[:, None] ** 2 * vis
+        var = w @ (vg * vg) - 2.0 * o * (w @ vg) + o * o * w.sum(axis=1)[:, None]
+        ds = (uq[:, h, :] @ np.abs(k8[:, g, :]).T + np.abs(q8[:, h, :]) @ uk[:, g, :].T) / np.sqrt(D)
+        O[:, h, :] = o
+        lse[:, h] = l_
+        sd[:, h, :] = np.sqrt(np.maximum(var, 0.0))
+        flip[:, h] = (p * ds).sum(axis=1)
+        if nk:
+            vdev[:, h, :] = np.where(live[:, None], np.abs(vg).max(axis=0)[None, :] + np.abs(o), 0.0)
+    return O, lse, sd, flip, vdev

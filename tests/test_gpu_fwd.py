@@ -1,6 +1,6 @@
 """GPU parity of the forward (CUDA path through the C ABI) against the fp64 oracle.
 
-Tolerances (stated with the benchmark spec of the method): O max-abs <= 1e-2 and
+Tolerances (those stated with the method's definition): O max-abs <= 1e-2 and
 mean-abs <= 1e-3, LSE max-abs <= 1e-3, on the same seeded bf16 inputs.  Small
 workloads are compared element by element over every row and head; full-size ones
 on a seeded row sample that always includes every slice edge."""

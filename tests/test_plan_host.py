@@ -181,3 +181,25 @@ def test_error_strings():
     for c in range(0, -10, -1):
         assert _abi.error_string(c) != "unknown error"
     assert _abi.error_string(-100) == "unknown error"
+
+
+def test_header_flag_and_error_constants_match_the_binding():
+    hdr = open(os.path.join(ROOT, "include", "bca.h")).read()
+    # plain numeric defines only (a value followed by a comment or the end of the line)
+    defs = dict(re.findall(r"^#define\s+(BCA_[A-Z0-9_]+)\s+\(?(-?(?:0x[0-9a-fA-F]+|\d+))u?\)?\s*(?:/\*.*)?$",
+                           hdr, flags=re.M))
+    for name, val in defs.items():
+        if hasattr(_abi, name):
+            assert getattr(_abi, name) == int(val, 0), name
+    for name in ("BCA_O_FP32", "BCA_PLAN_HOST_ONLY", "BCA_TEST_FORCE_TIMEOUT", "BCA_FWD_FP8_E4M3",
+                 "BCA_ERR_UNSUPPORTED"):
+        assert name in defs and hasattr(_abi, name), name
+
+
+def test_fp8_plan_compiles_on_host_and_refuses_the_backward():
+    w = W.WORKLOADS["tiny"]
+    p = Plan.from_workload(w, host_only=True, fp8=True)
+    assert p.info() == Plan.from_workload(w, host_only=True).info()
+    vp = [None] * 18                                      # every tensor pointer NULL
+    rc = p._lib.bca_bwd_ex(p._h, *vp, 0, None, None)
+    assert rc == _abi.BCA_ERR_UNSUPPORTED
