@@ -10,7 +10,8 @@ bound per element:
     |O_gpu - O_model| <= 6 sd + 2 flip * vdev + 2^-8 |O_model| + 1e-6
 (2^-8: bf16 output rounding), and |LSE_gpu - LSE_model| <= 2e-4 + 2 flip.  Against the
 exact fp64 oracle the e4m3 forward is only accurate to the format: the error is
-reported and bounded loosely (O within 0.1 absolute)."""
+reported and bounded loosely (O within 0.1 absolute on the workloads; with rows that see
+only a few keys, where one rounded V row can move O by 2^-4 of |V|, within 0.5)."""
 import numpy as np
 import pytest
 import torch
@@ -26,7 +27,7 @@ def _dev_inputs(w):
     return {k: (None if v is None else v.cuda()) for k, v in W.make_inputs(w, "cuda").items()}
 
 
-def _check(o_gpu, lse_gpu, model, exact, what):
+def _check(o_gpu, lse_gpu, model, exact, what, exact_bound=0.1):
     O8, L8, sd, flip, vdev = model
     o = o_gpu.double().cpu().numpy()
     l = lse_gpu.double().cpu().numpy().T
@@ -42,7 +43,7 @@ def _check(o_gpu, lse_gpu, model, exact, what):
            f"{el.max(initial=0):.3e}; vs exact O max {e_exact.max():.3e} mean {e_exact.mean():.3e}")
     assert worst <= 1.0, msg
     assert (el <= ltol).all(), msg
-    assert e_exact.max() <= 0.1, msg
+    assert e_exact.max() <= exact_bound, msg
     return msg
 
 
@@ -113,3 +114,34 @@ def test_fp8_is_deterministic_and_independent_of_bf16_plan():
     torch.cuda.synchronize()
     assert torch.equal(a, b) and torch.equal(la, lb8)
     assert not torch.equal(a, ob)                          # the e4m3 path did run
+
+
+def test_fp8_random_slices_with_empty_rows_and_causal():
+    """Overlapping FULL/CAUSAL slices with ragged, off-tile edges and rows that see
+    nothing (O = 0, LSE = -inf), each head dim, on the e4m3 path."""
+    rng = np.random.default_rng(15)
+    for trial in range(6):
+        nq = int(rng.integers(1, 400))
+        nc = int(rng.integers(0, 300))
+        nk = nq + nc
+        sl = []
+        for _ in range(int(rng.integers(0, 7))):
+            q0 = int(rng.integers(0, nq)); q1 = int(rng.integers(q0, nq + 1))
+            k0 = int(rng.integers(0, nk)); k1 = int(rng.integers(k0, nk + 1))
+            sl.append((q0, q1, k0, k1, int(rng.integers(0, 2))))
+        sl = np.asarray(sl, np.int64).reshape(-1, 5)
+        hq, hkv, d = 4, 2, (24, 32, 48)[trial % 3]
+        vids = np.asarray([[1, nq, 1, 1, 3]], np.int32)
+        seeds = 8000 + 10 * trial
+        q = W.seeded_normal_bf16(seeds, (nq, hq, d), "cuda")
+        k = W.seeded_normal_bf16(seeds + 1, (nq, hkv, d), "cuda")
+        v = W.seeded_normal_bf16(seeds + 2, (nq, hkv, d), "cuda")
+        kc = W.seeded_normal_bf16(seeds + 3, (nc, hkv, d), "cuda") if nc else None
+        vc = W.seeded_normal_bf16(seeds + 4, (nc, hkv, d), "cuda") if nc else None
+        p = Plan(hq, hkv, d, vids, nc, sl, o_fp32=bool(trial % 2), fp8=True)
+        o, lse = p.fwd(q, k, v, kc, vc)
+        torch.cuda.synchronize()
+        assert p.status() == 0
+        args = (q.cpu(), k.cpu(), v.cpu(), None if kc is None else kc.cpu(), None if vc is None else vc.cpu(),
+                vids, sl, hq, hkv)
+        print(_check(o, lse, oracle.forward_fp8(*args), oracle.forward(*args), f"trial {trial}", exact_bound=0.5))
