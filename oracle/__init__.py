@@ -369,10 +369,12 @@ def forward_fp8(q, k, v, k_cache, v_cache, videos, slices, hq, hkv,
     online softmax chooses (P <= 2^8), so its P differs from this P by a relative
     rounding error of at most 2^-4 per element in e4m3's normal range, and by at most
     2^-10 (half the subnormal step) in the kernel's P units below it, a unit at least
-    exp(lse - max s) in normalised probability.  Treating those errors as independent
-    and uniform gives the standard deviation returned as ``sd``:
+    exp(lse - max s) in normalised probability.  The row sum that normalises O is
+    formed from the unrounded fp32 P, so the errors do not cancel in the division:
+    O_gpu - O = sum_j p_ij e_ij v_jd.  Treating the e_ij as independent and uniform
+    gives the standard deviation returned as ``sd``:
         sd[i,h,d]^2 = sum_j ((2^-4/sqrt 3)^2 p_ij^2 + (2^-10/sqrt 3)^2 exp(2 (max_j s_ij - lse_i)))
-                      * (v_jd - o_id)^2.
+                      * v_jd^2.
     A Q-hat or K-hat element computed in fp32 (the kernel's prologue) within about 2e-6
     of an e4m3 rounding midpoint may round to the other neighbour, moving score s_ij by
     at most that element's step times its partner's magnitude / sqrt(D).  ``flip`` is
@@ -424,9 +426,8 @@ def forward_fp8(q, k, v, k_cache, v_cache, videos, slices, hq, hkv,
         p = ex / np.where(live, tot, 1.0)[:, None]
         vg = v8[:, g, :]
         o = p @ vg
-        # sum_j w_ij (v_jd - o_id)^2 = w@v^2 - 2 o (w@v) + o^2 sum_j w_ij
         w = (rel * p) ** 2 + (absu * np.where(live, np.exp(sm - l_), 0.0))[:, None] ** 2 * vis
-        var = w @ (vg * vg) - 2.0 * o * (w @ vg) + o * o * w.sum(axis=1)[:, None]
+        var = w @ (vg * vg)
         ds = (uq[:, h, :] @ np.abs(k8[:, g, :]).T + np.abs(q8[:, h, :]) @ uk[:, g, :].T) / np.sqrt(D)
         O[:, h, :] = o
         lse[:, h] = l_
