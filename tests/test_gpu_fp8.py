@@ -36,7 +36,7 @@ def _check(o_gpu, lse_gpu, model, exact, what, exact_bound=0.1):
     tol = 6 * sd + 2 * flip[:, :, None] * vdev + 2.0 ** -8 * np.abs(O8) + 1e-6
     err = np.abs(o - O8)
     worst = (err / tol).max()
-    el = np.abs(l - L8)[finite]
+    el = np.abs(np.where(finite, l, 0.0) - np.where(finite, L8, 0.0))[finite]
     ltol = (2e-4 + 2 * flip)[finite]
     e_exact = np.abs(o - exact[0])
     msg = (f"{what}: vs e4m3 model O max {err.max():.3e} (worst err/tol {worst:.2f}), LSE max "
