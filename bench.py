@@ -131,9 +131,13 @@ def _cpu_inputs(w):
     return _CPU_INPUTS[w.name]
 
 
-def cpu_oracle_sample(w, nrows: int, seed: int):
+def cpu_oracle_sample(w, nrows: int, seed: int, pass_: str = "fwd"):
     """Time the fp64 oracle (as it stands) on ``nrows`` seeded query rows, all heads.
-    Returns (seconds, mask-aware flops of the sample, description)."""
+    pass_ "fwd": the forward of those rows (S and P V: 4 D flops per visible pair and
+    head); "fwdbwd": the oracle's row backward, which recomputes the forward and forms
+    dP and dQ for those rows (S, P V, dO V^T, dS K: 8 D flops per pair and head; the
+    dK / dV shares of a row are not formed by the row oracle and are not counted).
+    Returns (seconds, flops of the sample, description)."""
     import oracle
     from block_causal_attention_b200 import workloads as W
     rows = np.random.default_rng(seed).choice(w.nq, size=nrows, replace=False)
@@ -141,13 +145,23 @@ def cpu_oracle_sample(w, nrows: int, seed: int):
     k, v, kc, vc = _cpu_inputs(w)
     q_rows = W.make_input_rows(w, W.T_Q, rows)
     pairs = sum(int(oracle.mask_row(w.slices_array(), w.nk, int(r)).sum()) for r in rows)
-    t0 = time.perf_counter()
-    oracle.forward(None, k, v, kc, vc, w.videos_array(), w.slices_array(), w.hq, w.hkv, base=w.rope_base,
-                   eps=w.eps, rows=rows, q_rows=q_rows)
-    dt = time.perf_counter() - t0
-    flops = 4.0 * w.d * w.hq * pairs
+    if pass_ == "fwdbwd":
+        do_rows = W.make_input_rows(w, W.T_DO, rows)
+        t0 = time.perf_counter()
+        oracle.backward_rows(q_rows, rows, k, v, kc, vc, do_rows, w.videos_array(), w.slices_array(), w.hq, w.hkv,
+                             base=w.rope_base, eps=w.eps)
+        dt = time.perf_counter() - t0
+        flops = 8.0 * w.d * w.hq * pairs
+        what = "forward and dQ backward (through the prologue)"
+    else:
+        t0 = time.perf_counter()
+        oracle.forward(None, k, v, kc, vc, w.videos_array(), w.slices_array(), w.hq, w.hkv, base=w.rope_base,
+                       eps=w.eps, rows=rows, q_rows=q_rows)
+        dt = time.perf_counter() - t0
+        flops = 4.0 * w.d * w.hq * pairs
+        what = "forward"
     desc = (f"{nrows} seeded query row(s) x all {w.hq} heads of {w.name} ({pairs} visible pairs/head), "
-            f"forward incl. the K prologue of all {w.nq} new keys, fp64")
+            f"{what} incl. the K prologue of all {w.nq} new keys, fp64")
     return dt, flops, desc
 
 
@@ -170,11 +184,11 @@ def run_reference(a):
     from block_causal_attention_b200 import workloads as W
     w = W.WORKLOADS[a.workload]
     for s in range(a.warmup):
-        cpu_oracle_sample(w, 1, 100 + s)
+        cpu_oracle_sample(w, 1, 100 + s, a.pass_)
     times, flops = [], []
     desc = ""
     for s in range(a.steps):
-        dt, fl, desc = cpu_oracle_sample(w, 1, 200 + s)
+        dt, fl, desc = cpu_oracle_sample(w, 1, 200 + s, a.pass_)
         times.append(dt)
         flops.append(fl)
     total_t = sum(times)
@@ -183,7 +197,7 @@ def run_reference(a):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": a.gpus,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * total_t / a.steps, "higher_is_better": True,
         "scaling": "strong", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "pass": "fwd", "sample_per_step": "1 query row x all heads"},
+        "config": {"workload": w.name, "pass": a.pass_, "sample_per_step": "1 query row x all heads"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -417,7 +431,7 @@ def run_ours(a):
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        dt, fl, desc = cpu_oracle_sample(w, a.cpu_rows, 1)
+        dt, fl, desc = cpu_oracle_sample(w, a.cpu_rows, 1, a.pass_)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle", "sample": desc,
                "seconds": dt}
 
