@@ -12,6 +12,10 @@
 //                     their Q tile into shared memory, run the online softmax on S
 //                     rows read from tensor memory, write P (bf16) for the second MMA,
 //                     and finish with O / l and the LSE.
+//   e4m3 variant    : the same kernel instantiated with F8 = true (plans created with
+//                     BCA_FWD_FP8_E4M3): v_amax_kernel finds max|V| per KV head,
+//                     kv_image8_kernel writes e4m3 K-hat and V / 2^e images, and the
+//                     MMAs run as kind::f8f6f4 with e4m3 Q-hat and P.
 //
 // The operation: attention restricted to the union of AttnSlices, with QK-Norm and
 // 3D RoPE applied to Q and K and 128/8 grouped query heads (MAGI-1 research notes
