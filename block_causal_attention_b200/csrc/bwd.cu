@@ -363,6 +363,9 @@ struct ItemCursor {
 };
 
 __device__ __forceinline__ bool wait_abort(uint32_t bar, uint32_t parity, int *status, volatile int *abort_flag) {
+    // A completed phase needs no look at the abort flag (a volatile shared load on every
+    // waiter's path); only a wait that would block has to know whether the CTA gives up.
+    if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (mbar_wait(bar, parity, kWaitTimeoutNs)) return true;
     atomicOr(status, kStatusTimeout);

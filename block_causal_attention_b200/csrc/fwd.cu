@@ -298,6 +298,10 @@ __device__ __forceinline__ void record_timeout(int *status, volatile int *abort_
 
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, int *status, volatile int *abort_flag,
                                               uint64_t timeout_ns = kWaitTimeoutNs) {
+    // A completed phase needs no look at the abort flag: the flag is a volatile shared
+    // load on every waiter's path (the MMA issuer waits several times per tile), and only
+    // a wait that would block has to know whether the CTA is giving up.
+    if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (mbar_wait(bar, parity, timeout_ns)) return true;
     record_timeout(status, abort_flag);
