@@ -145,3 +145,44 @@ def test_fp8_random_slices_with_empty_rows_and_causal():
         args = (q.cpu(), k.cpu(), v.cpu(), None if kc is None else kc.cpu(), None if vc is None else vc.cpu(),
                 vids, sl, hq, hkv)
         print(_check(o, lse, oracle.forward_fp8(*args), oracle.forward(*args), f"trial {trial}", exact_bound=0.5))
+
+
+def test_fp8_fwd_in_cuda_graph():
+    """The e4m3 forward (amax memset, amax and image kernels, attention) captured once in
+    a CUDA graph and replayed: bit-identical to eager launches, also after new V values
+    (the per-head scale is recomputed inside the graph)."""
+    w = W.WORKLOADS["b45_replica"]
+    x = _dev_inputs(w)
+    p = Plan.from_workload(w, fp8=True)
+    ws = p.alloc_workspace(_abi.BCA_PASS_FWD)
+    o = torch.empty((w.nq, w.hq, w.d), device="cuda", dtype=torch.bfloat16)
+    lse = torch.empty((w.hq, w.nq), device="cuda", dtype=torch.float32)
+    v = x["v"].clone()
+
+    def step():
+        p.fwd(x["q"], x["k"], v, x["k_cache"], x["v_cache"], o=o, lse=lse, workspace=ws)
+
+    step()
+    torch.cuda.synchronize()
+    ref_o, ref_l = o.clone(), lse.clone()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    o.zero_()
+    lse.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert p.status() == _abi.BCA_OK
+    assert torch.equal(o, ref_o) and torch.equal(lse, ref_l)
+    v.mul_(3.0)                                           # larger max|V|: a new scale exponent
+    g.replay()
+    eo, el = Plan.from_workload(w, fp8=True).fwd(x["q"], x["k"], v, x["k_cache"], x["v_cache"])
+    torch.cuda.synchronize()
+    assert torch.equal(o, eo) and torch.equal(lse, el)
+    del g
