@@ -4,6 +4,8 @@ covered exactly once).  No GPU needed: plans are built with BCA_PLAN_HOST_ONLY."
 import ctypes
 import os
 import re
+import subprocess
+import sys
 
 import numpy as np
 import pytest
@@ -203,3 +205,16 @@ def test_fp8_plan_compiles_on_host_and_refuses_the_backward():
     vp = [None] * 18                                      # every tensor pointer NULL
     rc = p._lib.bca_bwd_ex(p._h, *vp, 0, None, None)
     assert rc == _abi.BCA_ERR_UNSUPPORTED
+
+
+def test_missing_library_fails_loudly():
+    """With the native library absent the binding raises instead of falling back: there
+    is no CPU path behind Plan."""
+    code = ("import block_causal_attention_b200._abi as A, sys\n"
+            "A.LIB_PATH = '/nonexistent/libbca.so'\nA._lib = None\n"
+            "from block_causal_attention_b200 import Plan, workloads as W\n"
+            "try:\n    Plan.from_workload(W.WORKLOADS['tiny'], host_only=True)\n"
+            "except ImportError as e:\n    print('raised', e)\n    sys.exit(0)\n"
+            "sys.exit(1)\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and "raised" in r.stdout, r.stdout + r.stderr
