@@ -419,7 +419,9 @@ def run_ours(a):
             for line in f:
                 parts = line.split()
                 if len(parts) >= 3 and not parts[0].startswith("#") and parts[0] == dom and parts[1] == w.name:
-                    traffic = float(parts[2])
+                    # the line covers a launch over every KV group; this rank's launch runs
+                    # hkv of them (head-parallel shards), each with the same per-group work
+                    traffic = float(parts[2]) * hkv / w.hkv
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
                 "frac": achieved / peak_sus, "traffic": traffic,
                 "kernel": dom, "peak_kind": peak_kind,
