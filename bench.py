@@ -267,10 +267,20 @@ def run_ours(a):
             dist.barrier()
         torch.cuda.synchronize()
 
+    def any_rank_failed() -> bool:
+        """Device status of every rank, agreed by all (the same collective on every rank,
+        so a failure ends all ranks at once instead of leaving the others in a collective)."""
+        bad = plan.status() != 0
+        if world > 1:
+            t = torch.tensor([1.0 if bad else 0.0], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            bad = t.item() > 0
+        return bad
+
     for _ in range(a.warmup):
         step()
     barrier()
-    if plan.status() != 0:
+    if any_rank_failed():
         raise RuntimeError("device status error during warm-up")
 
     gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
@@ -289,7 +299,7 @@ def run_ours(a):
     prof = plan.profile_read()
     plan.profile(False)
     clk = clocks.stop()
-    if plan.status() != 0:
+    if any_rank_failed():
         raise RuntimeError("device status error in the timed region")
     if world > 1:
         t = torch.tensor([elapsed_ms], device="cuda", dtype=torch.float64)
