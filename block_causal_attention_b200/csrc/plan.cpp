@@ -150,7 +150,8 @@ int validate_problem(const bca_problem *p, Plan &P) {
         // packed RoPE positions: t - (smallest t0) < 65536, h, w < 256
         if (v.height > 256 || v.width > 256) return BCA_ERR_UNSUPPORTED;
         if ((int64_t)v.t0 + (int64_t)v.num_chunks * v.frames > INT32_MAX) return BCA_ERR_UNSUPPORTED;
-        nq += (int64_t)v.num_chunks * v.frames * v.height * v.width;
+        nq += (int64_t)v.num_chunks * v.frames * v.height * v.width;  // <= 2^47 per video
+        if (nq >= ((int64_t)1 << 31)) return BCA_ERR_UNSUPPORTED;      // checked per video: no wrap
     }
     P.nq = nq;
     P.nk = P.nc + nq;

@@ -164,6 +164,19 @@ def test_argument_checks_return_codes():
     assert _abi.lib().bca_plan_create(None, None) == E.BCA_ERR_INVALID_ARGUMENT
 
 
+
+def test_maximum_sizes_are_refused_before_any_allocation():
+    """Token counts past the 31-bit index space, frames past the 8-bit packed positions
+    and time positions past int32 are refused by validation (nothing is allocated)."""
+    E = _abi
+    assert _create(videos=((1, 1, 256, 256, 0),)) == E.BCA_OK                   # largest frame: 65,536 tokens
+    assert _create(videos=((1, 1, 4, 257, 0),)) == E.BCA_ERR_UNSUPPORTED        # width > 256
+    assert _create(videos=((32768, 1, 256, 256, 0),)) == E.BCA_ERR_UNSUPPORTED  # 2^31 tokens
+    assert _create(videos=((16384, 1, 256, 256, 0),) * 2) == E.BCA_ERR_UNSUPPORTED  # 2^30 + 2^30
+    assert _create(videos=((2, 1, 4, 4, 2 ** 31 - 2),)) == E.BCA_ERR_UNSUPPORTED    # t past int32
+    assert _create(videos=((2, 1, 4, 4, 0),), nc=2 ** 31 - 16) == E.BCA_ERR_UNSUPPORTED  # Nc + Nq = 2^31
+
+
 def test_host_only_plan_refuses_device_calls():
     p = _plan(W.WORKLOADS["tiny"])
     rc = _abi.lib().bca_fwd(p._h, *([None] * 11))
