@@ -19,9 +19,11 @@ answer on the dispatch solver gives the same cost model):
    ``k_prologue_bwd``); gradients of the global cache are summed over ranks.
 
 Every rank derives the whole dispatch from the same inputs, so no metadata is exchanged.
-Only FULL slices are handled (the slice language has no offset with which to cut a
-CAUSAL slice into shifted pieces); every workload of the pages is written with FULL
-slices.  The attention engine is pluggable: the default is this package's CUDA ``Plan``.
+CAUSAL slices (bottom-right aligned) are cut too: a causal slice restricted to a key
+sub-range [a, b) is exactly one CAUSAL band (the rows whose diagonal ends inside the
+range, with the band's own bottom-right corner on the diagonal) plus one FULL band (the
+rows that see all of [a, b)), and both forms survive the shift to local indices.
+The attention engine is pluggable: the default is this package's CUDA ``Plan``.
 """
 from __future__ import annotations
 
@@ -31,6 +33,7 @@ from typing import Callable, List, Optional, Sequence
 import numpy as np
 
 SLICE_FULL = 0
+SLICE_CAUSAL = 1
 
 
 @dataclasses.dataclass(frozen=True)
@@ -68,15 +71,50 @@ def _merge(iv):
     return [(a, b) for a, b in out]
 
 
+def causal_piece(q0: int, q1: int, k0: int, k1: int, qa: int, qb: int, a: int, b: int):
+    """The pairs of the CAUSAL slice (q0, q1, k0, k1) with rows in [qa, qb) and keys in
+    [a, b), as at most one CAUSAL and one FULL slice (same coordinates).
+
+    Bottom-right alignment: row i sees keys j in [k0, k1) with j - k0 <= (i - q0) +
+    (k1 - k0) - (q1 - q0), i.e. j < e(i) = i + k1 - q1 + 1.  Restricted to keys [lo, hi):
+    rows with e(i) <= lo see nothing, rows with e(i) >= hi see all of [lo, hi) (FULL),
+    and the rows between see [lo, e(i)): a CAUSAL slice whose bottom-right corner is
+    (last row, e(last row) - 1), so its own alignment gives the same e(i)."""
+    r0, r1 = max(q0, qa), min(q1, qb)
+    lo, hi = max(k0, a), min(k1, b)
+    if r0 >= r1 or lo >= hi:
+        return []
+    c = k1 - q1 + 1                               # e(i) = i + c
+    r_start = max(r0, lo - c + 1)                 # first row that sees a key of [lo, hi)
+    if r_start >= r1:
+        return []
+    r_full = min(r1, max(r_start, hi - c))        # first row that sees all of [lo, hi)
+    out = []
+    if r_start < r_full:
+        out.append((r_start, r_full, lo, r_full - 1 + c, SLICE_CAUSAL))
+    if r_full < r1:
+        out.append((r_full, r1, lo, hi, SLICE_FULL))
+    return out
+
+
+def _causal_of(slices, chunk: Chunk):
+    """The CAUSAL slices that reach the chunk's rows, as (q0, q1, k0, k1)."""
+    sl = np.asarray(slices, np.int64).reshape(-1, 5)
+    return [tuple(int(x) for x in r[:4]) for r in sl
+            if r[4] == SLICE_CAUSAL and max(int(r[0]), chunk.start) < min(int(r[1]), chunk.end)
+            and r[2] < r[3]]
+
+
 def chunk_rows(slices, chunk: Chunk, nc: int):
-    """Row groups of a chunk with their merged visible key intervals: a list of
-    (q_begin, q_end, [(k_begin, k_end), ...]) in global query / key indices."""
+    """Row groups of a chunk with the merged key intervals of its FULL slices: a list of
+    (q_begin, q_end, [(k_begin, k_end), ...]) in global query / key indices.  CAUSAL
+    slices are taken separately (``_causal_of``)."""
     sl = np.asarray(slices, np.int64).reshape(-1, 5)
     cuts = {chunk.start, chunk.end}
     mine = []
     for q0, q1, k0, k1, t in sl:
         if t != SLICE_FULL:
-            raise NotImplementedError("context parallelism handles FULL slices only")
+            continue
         a, b = max(int(q0), chunk.start), min(int(q1), chunk.end)
         if a < b and k0 < k1:
             mine.append((a, b, int(k0), int(k1)))
@@ -90,8 +128,29 @@ def chunk_rows(slices, chunk: Chunk, nc: int):
     return groups
 
 
+def _row_intervals(groups, causal, chunk: Chunk):
+    """Per row of the chunk, the merged visible key intervals of its FULL row groups and
+    its CAUSAL slices (used only when the chunk has CAUSAL slices)."""
+    per = [[] for _ in range(chunk.end - chunk.start)]
+    for a, b, iv in groups:
+        for i in range(a, b):
+            per[i - chunk.start].extend(iv)
+    for q0, q1, k0, k1 in causal:
+        c = k1 - q1 + 1
+        for i in range(max(q0, chunk.start), min(q1, chunk.end)):
+            e = min(k1, i + c)
+            if e > k0:
+                per[i - chunk.start].append((k0, e))
+    return [_merge(x) for x in per]
+
+
 def chunk_area(slices, chunk: Chunk, nc: int) -> int:
-    return sum((b - a) * sum(k1 - k0 for k0, k1 in iv) for a, b, iv in chunk_rows(slices, chunk, nc))
+    """Visible (query, key) pairs of the chunk's rows (the union over all slices)."""
+    groups = chunk_rows(slices, chunk, nc)
+    causal = _causal_of(slices, chunk)
+    if not causal:
+        return sum((b - a) * sum(k1 - k0 for k0, k1 in iv) for a, b, iv in groups)
+    return sum(k1 - k0 for row in _row_intervals(groups, causal, chunk) for k0, k1 in row)
 
 
 def dispatch(chunks: Sequence[Chunk], areas: Sequence[int], world: int) -> List[int]:
@@ -115,7 +174,7 @@ class LocalProblem:
     videos: np.ndarray           # [n_chunks, 5] single-chunk videos
     cache_rows: np.ndarray       # global cache rows needed, sorted
     remote_rows: np.ndarray      # global token indices of borrowed keys, sorted
-    slices: np.ndarray           # [m, 5] local FULL slices
+    slices: np.ndarray           # [m, 5] local slices (FULL and CAUSAL)
     area: int
     slices_held: np.ndarray      # the slices restricted to keys held locally: keys [cache rows | own]
     slices_borrowed: np.ndarray  # restricted to borrowed keys: keys [borrowed rows | own (unused)]
@@ -134,7 +193,8 @@ class ContextParallelPlan:
         self.chunks = chunks_of(videos)
         self.nq = self.chunks[-1].end if self.chunks else 0
         self.rows = [chunk_rows(slices, c, self.nc) for c in self.chunks]
-        self.areas = [sum((b - a) * sum(k1 - k0 for k0, k1 in iv) for a, b, iv in g) for g in self.rows]
+        self.causal = [_causal_of(slices, c) for c in self.chunks]
+        self.areas = [self._area(i) for i in range(len(self.chunks))]
         self.owner = dispatch(self.chunks, self.areas, self.world)
         self.token_owner = np.zeros(self.nq, np.int64)
         for c, r in zip(self.chunks, self.owner):
@@ -147,6 +207,14 @@ class ContextParallelPlan:
             own = self.token_owner[rr] if len(rr) else np.zeros(0, np.int64)
             for src in range(self.world):
                 self.send_rows[src][dst] = rr[own == src]
+
+    def _area(self, i: int) -> int:
+        """Visible pairs of chunk i's rows: the union of its FULL row groups and CAUSAL
+        slices (per row only when the chunk has CAUSAL slices)."""
+        if not self.causal[i]:
+            return sum((b - a) * sum(k1 - k0 for k0, k1 in iv) for a, b, iv in self.rows[i])
+        return sum(k1 - k0 for row in _row_intervals(self.rows[i], self.causal[i], self.chunks[i])
+                   for k0, k1 in row)
 
     def _local(self, r: int) -> LocalProblem:
         mine = [i for i, o in enumerate(self.owner) if o == r]
@@ -163,6 +231,9 @@ class ContextParallelPlan:
             for a, b, iv in self.rows[i]:
                 for k0, k1 in iv:
                     need[k0:k1] = True
+            c = self.chunks[i]
+            for q0, q1, k0, k1 in self.causal[i]:   # rows see [k0, e(i)), e growing with i
+                need[k0:min(k1, min(q1, c.end) - 1 + k1 - q1 + 1)] = True
         need &= ~own
         cache_rows = np.flatnonzero(need[:self.nc]).astype(np.int64)
         remote_rows = np.flatnonzero(need[self.nc:]).astype(np.int64)
@@ -172,21 +243,32 @@ class ContextParallelPlan:
         lk[cache_rows] = np.arange(len(cache_rows))
         lk[self.nc + remote_rows] = len(cache_rows) + np.arange(len(remote_rows))
         lk[self.nc + tokens] = nc_loc + np.arange(len(tokens))
+        def runs(k0, k1):
+            """Maximal runs of global keys [k0, k1) whose local index advances by one:
+            (global start, global end, local start)."""
+            seg = lk[k0:k1]
+            cuts = np.flatnonzero(np.diff(seg) != 1) + 1
+            starts = np.concatenate([[0], cuts])
+            ends = np.concatenate([cuts, [k1 - k0]])
+            return [(k0 + int(s0), k0 + int(s1), int(seg[s0])) for s0, s1 in zip(starts, ends)]
+
         out = []
         area = 0
         for ci, i in enumerate(mine):
             c = self.chunks[i]
+            dq = first_local[ci] - c.start                # global row -> local row
+            area += self.areas[i]
             for a, b, iv in self.rows[i]:
-                qa, qb = a - c.start + first_local[ci], b - c.start + first_local[ci]
                 for k0, k1 in iv:
-                    area += (b - a) * (k1 - k0)
-                    seg = lk[k0:k1]
-                    # pieces: maximal runs where the local index advances by one
-                    cuts = np.flatnonzero(np.diff(seg) != 1) + 1
-                    starts = np.concatenate([[0], cuts])
-                    ends = np.concatenate([cuts, [k1 - k0]])
-                    for s0, s1 in zip(starts, ends):
-                        out.append((qa, qb, int(seg[s0]), int(seg[s0]) + int(s1 - s0), SLICE_FULL))
+                    for ga, gb, la in runs(k0, k1):
+                        out.append((a + dq, b + dq, la, la + gb - ga, SLICE_FULL))
+            for q0, q1, k0, k1 in self.causal[i]:
+                e_last = min(k1, min(q1, c.end) - 1 + k1 - q1 + 1)
+                if e_last <= k0:
+                    continue
+                for ga, gb, la in runs(k0, e_last):
+                    for ra, rb, ka, kb, t in causal_piece(q0, q1, k0, k1, c.start, c.end, ga, gb):
+                        out.append((ra + dq, rb + dq, ka - ga + la, kb - ga + la, t))
         sl = np.asarray(out, np.int64).reshape(-1, 5)
         # split at the region boundaries: [0, ncache) cache, [ncache, nc_loc) borrowed, own
         ncache, nrem = len(cache_rows), len(remote_rows)
@@ -194,9 +276,13 @@ class ContextParallelPlan:
         for qa, qb, k0, k1, t in out:
             for lo, hi, dst, shift in ((0, ncache, held, 0), (ncache, nc_loc, borrowed, -ncache),
                                        (nc_loc, nc_loc + len(tokens), held, -nrem)):
-                a0, a1 = max(k0, lo), min(k1, hi)
-                if a0 < a1:
-                    dst.append((qa, qb, a0 + shift, a1 + shift, t))
+                if t == SLICE_FULL:
+                    a0, a1 = max(k0, lo), min(k1, hi)
+                    if a0 < a1:
+                        dst.append((qa, qb, a0 + shift, a1 + shift, t))
+                else:
+                    for ra, rb, ka, kb, tt in causal_piece(qa, qb, k0, k1, qa, qb, lo, hi):
+                        dst.append((ra, rb, ka + shift, kb + shift, tt))
         sh = np.asarray(held, np.int64).reshape(-1, 5)
         sb = np.asarray(borrowed, np.int64).reshape(-1, 5)
         return LocalProblem(r, mine, tokens, videos, cache_rows, remote_rows, sl, area, sh, sb)

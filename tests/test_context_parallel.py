@@ -52,9 +52,66 @@ def test_dispatch_balances_area():
     assert max(load) - min(load) <= 1 and sum(load) == sum(areas)
 
 
-def test_causal_slices_are_rejected():
-    with pytest.raises(NotImplementedError):
-        CP.ContextParallelPlan(2, [[2, 1, 2, 2, 0]], 0, [[0, 8, 0, 8, 1]])
+def test_causal_piece_equals_the_restricted_slice_by_brute_force():
+    """A CAUSAL slice restricted to rows [qa, qb) and keys [a, b) is exactly the union of
+    the returned pieces (pair by pair), and the pieces do not overlap."""
+    rng = np.random.default_rng(7)
+    for _ in range(3000):
+        n, m = int(rng.integers(1, 24)), int(rng.integers(1, 24))
+        q0 = int(rng.integers(0, n)); q1 = int(rng.integers(q0, n + 1))
+        k0 = int(rng.integers(0, m)); k1 = int(rng.integers(k0, m + 1))
+        qa = int(rng.integers(0, n)); qb = int(rng.integers(qa, n + 1))
+        a = int(rng.integers(0, m)); b = int(rng.integers(a, m + 1))
+        want = oracle.mask_dense(np.asarray([[q0, q1, k0, k1, 1]], np.int64), n, m).astype(bool)
+        want[:qa] = want[qb:] = False
+        want[:, :a] = want[:, b:] = False
+        got = np.zeros((n, m), np.int32)
+        for piece in CP.causal_piece(q0, q1, k0, k1, qa, qb, a, b):
+            got += oracle.mask_dense(np.asarray([piece], np.int64), n, m)
+        assert got.max(initial=0) <= 1 and np.array_equal(got.astype(bool), want), (q0, q1, k0, k1, qa, qb, a, b)
+
+
+def _random_slices(rng, nq, nk, count):
+    sl = []
+    for _ in range(count):
+        q0 = int(rng.integers(0, nq)); q1 = int(rng.integers(q0 + 1, nq + 1))
+        k0 = int(rng.integers(0, nk)); k1 = int(rng.integers(k0 + 1, nk + 1))
+        sl.append((q0, q1, k0, k1, int(rng.integers(0, 2))))
+    return np.asarray(sl, np.int64).reshape(-1, 5)
+
+
+@pytest.mark.parametrize("seed", range(8))
+@pytest.mark.parametrize("world", [1, 2, 3])
+def test_local_problems_reproduce_random_full_and_causal_masks(seed, world):
+    """Random overlapping FULL and CAUSAL slices over a cache and several chunks: the
+    ranks' local masks (and their held / borrowed splits) map back onto the global mask
+    exactly, each query row on one rank."""
+    rng = np.random.default_rng(100 + seed)
+    nchunks, nc = int(rng.integers(2, 6)), int(rng.integers(0, 20))
+    vid = np.asarray([[nchunks, 1, 2, 4, 0]], np.int32)          # chunks of 8 tokens
+    nq = nchunks * 8
+    sl = _random_slices(rng, nq, nc + nq, int(rng.integers(1, 7)))
+    cp = CP.ContextParallelPlan(world, vid, nc, sl)
+    ref = oracle.mask_dense(sl, nq, nc + nq).astype(bool)
+    union = np.zeros_like(ref)
+    for r in range(world):
+        lm = _local_mask(cp, r)
+        assert not (union & lm).any()
+        union |= lm
+        assert cp.local[r].area == int(lm.sum())
+        lp = cp.local[r]
+        nql, ncache, nrem = len(lp.tokens), len(lp.cache_rows), len(lp.remote_rows)
+        g = np.zeros_like(ref)
+        for sls, keys in ((lp.slices_held, np.concatenate([lp.cache_rows, nc + lp.tokens])),
+                          (lp.slices_borrowed, np.concatenate([nc + lp.remote_rows, nc + lp.tokens]))):
+            m = oracle.mask_dense(sls, nql, len(keys)).astype(bool) if nql else np.zeros((0, len(keys)), bool)
+            qi, kj = np.nonzero(m)
+            part = np.zeros_like(ref)
+            part[lp.tokens[qi], keys[kj].astype(np.int64)] = True
+            assert not (g & part).any()                      # held and borrowed do not overlap
+            g |= part
+        assert np.array_equal(g, lm)
+    assert np.array_equal(union, ref)
 
 
 # --------------------------------------------------------------------------- gloo ranks
@@ -144,8 +201,27 @@ def _small_cached():
                            eps=1e-6, videos_array=lambda: vid, slices_array=lambda: sl)
 
 
+def _small_causal():
+    """A cache of 24 keys and 3 query chunks of 16 tokens with overlapping FULL and
+    CAUSAL slices, including causal slices with |q| != |k| (bottom-right aligned)."""
+    from types import SimpleNamespace
+    C, nc = 16, 24
+    sl = np.asarray([[0, 48, 0, nc, 0],                  # every query sees the cache
+                     [0, 48, nc, nc + 48, 1],            # token-causal over the new tokens
+                     [16, 32, nc, nc + 16, 0],           # chunk 1 also sees chunk 0 fully
+                     [32, 48, 8, nc + 40, 1],            # |q| = 16, |k| = 56: bottom-right aligned
+                     [20, 28, 0, 6, 1]], np.int64)       # |q| = 8 > |k| = 6: early rows see nothing
+    vid = np.asarray([[3, 1, 4, 4, 0]], np.int32)
+    return SimpleNamespace(nq=3 * C, nk=nc + 3 * C, hq=4, hkv=2, d=24, num_cache_keys=nc, rope_base=(50.0, 30.0, 20.0),
+                           eps=1e-6, videos_array=lambda: vid, slices_array=lambda: sl)
+
+
 def _workload(name):
-    return _small_cached() if name == "small_cached" else W.WORKLOADS[name]
+    if name == "small_cached":
+        return _small_cached()
+    if name == "small_causal":
+        return _small_causal()
+    return W.WORKLOADS[name]
 
 
 def _inputs(w):
@@ -192,7 +268,8 @@ def _free_port():
 
 @pytest.mark.parametrize("name,world,overlap", [("b45_replica", 2, False), ("packed_replica", 3, False),
                                                 ("kvrange_replica", 2, True), ("tiny", 3, True),
-                                                ("small_cached", 2, False), ("small_cached", 3, True)])
+                                                ("small_cached", 2, False), ("small_cached", 3, True),
+                                                ("small_causal", 2, False), ("small_causal", 3, True)])
 def test_gloo_ranks_match_the_single_process_oracle(name, world, overlap, tmp_path):
     """overlap=True: each rank attends to the keys it holds while the borrowed ones are in
     flight and merges the two partial results by their log-sum-exps."""
