@@ -167,3 +167,22 @@ def test_bwd_full_size_sampled_dq_and_dv_sums(name, nrows):
     # P enters dV rounded to bf16 (relative 2^-9 per element), so the identity holds to
     # about that precision, not to fp32 rounding
     assert rel < 1e-2, rel
+
+
+@pytest.mark.parametrize("name,groups", [("b45_infer", (0, 5))])
+def test_bwd_full_size_sampled_key_rows(name, groups):
+    """Full size, in the benchmark's launch configuration: dK (w.r.t. the raw keys) and dV
+    of seeded key rows of the last two chunks, for two KV groups, computed exactly by the
+    oracle from only the query rows that see those keys (tests/packed_keys.py)."""
+    import sys, os
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+    from packed_keys import video_key_grads, video_span
+    w = W.WORKLOADS[name]
+    x = W.make_inputs(w, "cuda", with_grad=True)
+    dq, dk, dv, dkc, dvc = _gpu_fwd_bwd(w, x)
+    start, C, nch = video_span(w, 0)
+    keys = np.sort(np.random.default_rng(11).choice(np.arange((nch - 2) * C, nch * C), 96, replace=False))
+    kr = torch.as_tensor(start + keys, device="cuda")
+    for g in groups:
+        rk, rv = video_key_grads(w, 0, g, keys)
+        print(name, g, _err("dk rows", dk[kr, g], rk), _err("dv rows", dv[kr, g], rv))

@@ -374,3 +374,22 @@ def test_backward_dv_sums_to_do_sum():
     for g in range(Hkv):
         assert np.allclose(dv[:, g].sum(0), do[:, 2 * g:2 * g + 2].sum((0, 1)), atol=1e-10)
         assert np.allclose(dk[:, g].sum(0), 0, atol=1e-10)
+
+
+def test_video_key_grads_equal_the_dense_backward():
+    """The per-video key-row helper of the full-size backward checks (packed_keys) gives
+    the dense oracle backward's dK and dV, for videos of a packed workload and each group."""
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+    from packed_keys import video_key_grads, video_span
+    w = W.WORKLOADS["packed_replica"]
+    x = W.make_inputs(w, "cpu", with_grad=True)
+    _, dk, dv, _, _, _, _ = oracle.backward(x["q"], x["k"], x["v"], None, None, x["do"], w.videos_array(),
+                                            w.slices_array(), w.hq, w.hkv, base=w.rope_base, eps=w.eps)
+    for vi in (1, 2):
+        start, C, nch = video_span(w, vi)
+        keys = np.unique(np.random.default_rng(vi).integers(max(0, nch - 2) * C, nch * C, 40))
+        for g in range(w.hkv):
+            k_dk, k_dv = video_key_grads(w, vi, g, keys)
+            assert np.abs(k_dk - dk[start + keys, g]).max() <= 1e-12
+            assert np.abs(k_dv - dv[start + keys, g]).max() <= 1e-12
