@@ -445,7 +445,9 @@ def run_ours(a):
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         dt, fl, desc = cpu_oracle_sample(w, a.cpu_rows, 1, a.pass_)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle", "sample": desc,
-               "seconds": dt}
+               "seconds": dt,
+               # extrapolated, not measured: one whole step of this workload at the sample's rate
+               "extrapolated_step_seconds": flops_step_total / (fl / dt)}
 
     if rank == 0:
         line = {

@@ -162,6 +162,26 @@ def test_prologue_zero_position_is_plain_rms_norm():
     assert np.allclose(y, g * x / rms, rtol=1e-13, atol=0)
 
 
+@pytest.mark.parametrize("D", [24, 48])
+def test_prologue_huge_base_leaves_only_the_first_pair_of_each_axis_rotating(D):
+    """Pair k of an axis rotates by pos * base^(-k/p): as the base grows every pair but
+    the first (k = 0, frequency 1 for any base) stops rotating, so the output is the plain
+    RMS norm except channels (0, 1) of each axis segment, rotated by that axis's position."""
+    p = (D // 2) // 3
+    x = _rand((6, 1, D))
+    pos = np.asarray([[3, 1, 2], [0, 5, 7], [9, 0, 0], [1, 1, 1], [4, 2, 6], [2, 3, 0]], np.int32)
+    y = oracle.prologue(x, pos, base=(1e300, 1e300, 1e300), eps=1e-6)
+    z = x / np.sqrt((x ** 2).mean(-1, keepdims=True) + 1e-6)
+    want = z.copy()
+    for a in range(3):
+        c0 = 2 * p * a
+        th = pos[:, a].astype(np.float64)[:, None]
+        x0, x1 = z[:, :, c0], z[:, :, c0 + 1]
+        want[:, :, c0] = x0 * np.cos(th) - x1 * np.sin(th)
+        want[:, :, c0 + 1] = x0 * np.sin(th) + x1 * np.cos(th)
+    assert np.allclose(y, want, rtol=0, atol=1e-12)
+
+
 @pytest.mark.parametrize("D", [24, 32, 48])
 def test_prologue_rope_pairs_are_adjacent_channels(D):
     """A basis vector on channel 2k of axis a rotates into channel 2k+1 of the same
