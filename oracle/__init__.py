@@ -359,6 +359,10 @@ def forward_fp8(q, k, v, k_cache, v_cache, videos, slices, hq, hkv,
                 base=(1e4, 1e4, 1e4), eps=1e-6, q_gain=None, k_gain=None, rows=None, q_rows=None):
     """The forward with e4m3 operands, and the spread its last rounding leaves.
 
+    FP8 on the pages: MAGI-1 research notes, inference infrastructure (real-time streaming
+    scenario): the linear layers run W8A8 in FP8 (SmoothQuant).  The attention variant
+    modelled here puts the same 8-bit format on the attention operands.
+
     Same method as ``forward`` with the tensor-core operands rounded to e4m3: Q-hat and
     K-hat after the prologue (unscaled; the softmax scale 1/sqrt(D) multiplies the
     fp64 score), and V divided by 2^e per KV head (``e4m3_scale_exponent`` of max|V|
