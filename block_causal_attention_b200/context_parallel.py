@@ -348,6 +348,40 @@ class ContextParallelAttention:
             self.plan_borrowed = eng(hq, hkv, d, lp.videos, len(lp.remote_rows), lp.slices_borrowed, rope_base, eps,
                                      True)
         self._saved = None
+        self._index_maps()
+        self._dev_idx = {}
+
+    def _index_maps(self):
+        """Row indices of the exchanges, fixed by the dispatch (``local.tokens`` and
+        ``local.remote_rows`` are sorted, so every lookup is a binary search):
+        - send_idx[dst]: rows of this rank's tokens that dst borrows (its K-hat / V);
+        - recv_order: for each borrowed row, in remote_rows order, its place in the
+          concatenated receive buffer (sources in rank order, each in global order);
+        - ret_send_idx[dst]: rows of remote_rows that belong to dst (their gradients);
+        - ret_recv_idx[src]: rows of this rank's tokens that src returns gradients for."""
+        cp, r, lp = self.cp, self.rank, self.local
+        tok, rr = lp.tokens.astype(np.int64), lp.remote_rows.astype(np.int64)
+        self.send_idx = [np.searchsorted(tok, cp.send_rows[r][dst]) for dst in range(self.world)]
+        self.recv_counts = [len(cp.send_rows[src][r]) for src in range(self.world)]
+        own = cp.token_owner[rr] if len(rr) else np.zeros(0, np.int64)
+        offs = np.cumsum([0] + self.recv_counts)
+        j = np.zeros(len(rr), np.int64)
+        for src in range(self.world):
+            m = own == src
+            j[m] = np.arange(int(m.sum()))
+        self.recv_order = (offs[own] + j) if len(rr) else np.zeros(0, np.int64)
+        self.ret_send_idx = [np.searchsorted(rr, cp.send_rows[dst][r]) for dst in range(self.world)]
+        self.ret_recv_idx = [np.searchsorted(tok, cp.send_rows[r][src]) for src in range(self.world)]
+
+    def _idx(self, name, arr, device):
+        """The index array as a torch tensor on the device (made once per device)."""
+        import torch
+        key = (name, str(device))
+        t = self._dev_idx.get(key)
+        if t is None:
+            t = torch.as_tensor(arr, dtype=torch.long, device=device)
+            self._dev_idx[key] = t
+        return t
 
     def _gather_keys(self, khat_local, v_local):
         return self._gather_keys_finish(self._gather_keys_start(khat_local, v_local))
@@ -356,15 +390,10 @@ class ContextParallelAttention:
         """Send the rows of [K-hat | V] of this rank's tokens that the other ranks need;
         returns a handle for _gather_keys_finish (the receive may still be in flight)."""
         import torch
-        cp, r = self.cp, self.rank
-        pos_in_local = {int(t): j for j, t in enumerate(self.local.tokens)}
         kv = torch.stack([khat_local, v_local], 1)                      # [n, 2, Hkv, D]
-        send = []
-        for dst in range(self.world):
-            rows = cp.send_rows[r][dst]
-            idx = torch.as_tensor([pos_in_local[int(t)] for t in rows], dtype=torch.long, device=kv.device)
-            send.append(kv.index_select(0, idx))
-        recv_counts = [len(cp.send_rows[src][r]) for src in range(self.world)]
+        send = [kv.index_select(0, self._idx(("send", dst), self.send_idx[dst], kv.device))
+                for dst in range(self.world)]
+        recv_counts = self.recv_counts
         return _all_to_all_rows(self.group, send, recv_counts, kv.shape[1:], kv, async_op=True), recv_counts, kv
 
     def _gather_keys_finish(self, handle):
@@ -373,19 +402,10 @@ class ContextParallelAttention:
         (got, work), recv_counts, kv = handle
         if work is not None:
             work.wait()
-        cp, r = self.cp, self.rank
         # reorder to local.remote_rows: each source sent its subset in global order
-        rr = self.local.remote_rows
-        order = {}
-        for src in range(self.world):
-            for j, t in enumerate(cp.send_rows[src][r]):
-                order[int(t)] = (src, j)
-        if len(rr):
+        if len(self.local.remote_rows):
             cat = torch.cat(got, 0)
-            offs = np.cumsum([0] + recv_counts)
-            idx = torch.as_tensor([offs[order[int(t)][0]] + order[int(t)][1] for t in rr], dtype=torch.long,
-                                  device=kv.device)
-            rem = cat.index_select(0, idx)
+            rem = cat.index_select(0, self._idx("recv", self.recv_order, kv.device))
         else:
             rem = kv.new_zeros((0,) + tuple(kv.shape[1:]))
         return rem[:, 0], rem[:, 1]
@@ -412,12 +432,8 @@ class ContextParallelAttention:
         import torch
         cp, r = self.cp, self.rank
         grads = torch.stack([rem_k, rem_v], 1)                             # [n_remote, 2, Hkv, D]
-        rpos = {int(t): j for j, t in enumerate(self.local.remote_rows)}
-        send = []
-        for dst in range(self.world):
-            idx = torch.as_tensor([rpos[int(t)] for t in cp.send_rows[dst][r]], dtype=torch.long,
-                                  device=grads.device)
-            send.append(grads.index_select(0, idx))
+        send = [grads.index_select(0, self._idx(("ret_send", dst), self.ret_send_idx[dst], grads.device))
+                for dst in range(self.world)]
         recv_counts = [len(cp.send_rows[r][src]) for src in range(self.world)]
         return _all_to_all_rows(self.group, send, recv_counts, grads.shape[1:], grads, async_op=True)
 
@@ -427,13 +443,10 @@ class ContextParallelAttention:
         got, work = handle
         if work is not None:
             work.wait()
-        cp, r = self.cp, self.rank
-        pos_in_local = {int(t): j for j, t in enumerate(self.local.tokens)}
         dkh = dk.new_zeros(dk.shape)
         for src in range(self.world):
-            rows = cp.send_rows[r][src]
-            if len(rows):
-                idx = torch.as_tensor([pos_in_local[int(t)] for t in rows], dtype=torch.long, device=dk.device)
+            if len(self.ret_recv_idx[src]):
+                idx = self._idx(("ret_recv", src), self.ret_recv_idx[src], dk.device)
                 dkh.index_add_(0, idx, got[src][:, 0])
                 dv.index_add_(0, idx, got[src][:, 1])
         dk = self.plan.k_prologue_bwd(k_local, dkh, k_gain, dk=dk, accumulate=True)
