@@ -269,7 +269,8 @@ def _free_port():
 @pytest.mark.parametrize("name,world,overlap", [("b45_replica", 2, False), ("packed_replica", 3, False),
                                                 ("kvrange_replica", 2, True), ("tiny", 3, True),
                                                 ("small_cached", 2, False), ("small_cached", 3, True),
-                                                ("small_causal", 2, False), ("small_causal", 3, True)])
+                                                ("small_causal", 1, False), ("small_causal", 2, False),
+                                                ("small_causal", 3, True)])
 def test_gloo_ranks_match_the_single_process_oracle(name, world, overlap, tmp_path):
     """overlap=True: each rank attends to the keys it holds while the borrowed ones are in
     flight and merges the two partial results by their log-sum-exps."""
