@@ -169,7 +169,9 @@ int bca_plan_expand_cols(bca_plan_t plan, int64_t key_begin, int64_t key_end, ui
  * BCA_ERR_INVALID_ARGUMENT for a changed geometry or a negative t0. */
 int bca_plan_update_positions(bca_plan_t plan, const bca_video *videos, int num_videos, void *stream);
 
-/* Bytes of caller-provided device workspace a pass needs (16-byte aligned). */
+/* Bytes of caller-provided device workspace a pass needs (16-byte aligned).  The
+ * forward's size covers both operand formats: the bf16/fp16 tile images, or for
+ * BCA_FWD_FP8_E4M3 plans the smaller e4m3 images plus one float of max|V| per KV head. */
 size_t bca_workspace_bytes(bca_plan_t plan, int pass);
 
 /* Forward.  q, k, v, k_cache, v_cache: bf16 (k_cache/v_cache NULL iff Nc == 0);
