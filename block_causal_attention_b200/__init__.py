@@ -228,6 +228,12 @@ class Plan:
             self._lib.bca_plan_destroy(self._h)
             self._h = _abi.ctypes.c_void_p()
 
+    def __enter__(self) -> "Plan":
+        return self
+
+    def __exit__(self, *exc) -> None:
+        self.close()
+
     def __del__(self):
         try:
             self.close()

@@ -231,3 +231,10 @@ def test_missing_library_fails_loudly():
             "sys.exit(1)\n")
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and "raised" in r.stdout, r.stdout + r.stderr
+
+
+def test_plan_is_a_context_manager_and_close_is_idempotent():
+    with Plan.from_workload(W.WORKLOADS["tiny"], host_only=True) as p:
+        assert p.info()["num_q"] == 192
+    assert not p._h.value                       # destroyed on exit
+    p.close()                                   # a second close is a no-op
