@@ -52,7 +52,7 @@ int upload(bca::Plan &P) {
     const size_t s_coloff = round256(P.col_off.size() * sizeof(int32_t));
     const size_t s_colruns = round256(std::max<size_t>(1, P.col_runs.size()) * sizeof(Run));
     const size_t s_bitems = round256(std::max<size_t>(1, P.bwd_items.size()) * sizeof(int32_t));
-    const size_t s_status = 256;
+    const size_t s_status = 256;  // the status word, then rope_tbase at byte 128
     const size_t total = s_runoff + s_runs + s_masks + s_items + s_pos + s_rope + s_coloff + s_colruns +
                          s_bitems + s_status;
     if (cudaGetDevice(&P.device) != cudaSuccess) return BCA_ERR_CUDA;
@@ -78,10 +78,13 @@ int upload(bca::Plan &P) {
     P.d_bwd_items =
         static_cast<const int32_t *>(put(P.bwd_items.data(), P.bwd_items.size() * sizeof(int32_t), s_bitems));
     P.d_status = static_cast<int *>(static_cast<void *>(b + off));
+    P.d_tbase = static_cast<int32_t *>(static_cast<void *>(b + off + 128));
     if (!P.d_run_off || !P.d_runs || !P.d_masks || !P.d_items || !P.d_pos || !P.d_rope || !P.d_col_off ||
         !P.d_col_runs || !P.d_bwd_items)
         return BCA_ERR_CUDA;
     if (cudaMemset(P.d_status, 0, sizeof(int)) != cudaSuccess) return BCA_ERR_CUDA;
+    if (cudaMemcpy(P.d_tbase, &P.rope_tbase, sizeof(int32_t), cudaMemcpyHostToDevice) != cudaSuccess)
+        return BCA_ERR_CUDA;
     P.rope_capacity = P.rope.size();
     int rc = prepare_fwd(P);
     if (rc == BCA_OK) rc = prepare_bwd(P);
@@ -144,19 +147,20 @@ int bca_plan_update_positions(bca_plan_t plan, const bca_video *videos, int num_
     for (int a = 0; a < 3; ++a) next.base[a] = P.base[a];
     int rc;
     try {
-        rc = bca::build_positions(next);
+        // on the device the table keeps the plan's layout (a t range that grew does not fit)
+        rc = bca::build_positions(next, on_device ? &P : nullptr);
     } catch (const std::bad_alloc &) {
         rc = BCA_ERR_NO_MEMORY;
     }
     if (rc != BCA_OK) return rc;
-    if (on_device && next.rope.size() > P.rope_capacity) return BCA_ERR_UNSUPPORTED;  // the t range grew
     if (on_device) {
         cudaStream_t s = static_cast<cudaStream_t>(stream);
         // pageable sources: the copies are staged before return, ordered on the stream
         if (cudaMemcpyAsync(const_cast<uint32_t *>(P.d_pos), next.pos.data(), next.pos.size() * sizeof(uint32_t),
                             cudaMemcpyHostToDevice, s) != cudaSuccess ||
             cudaMemcpyAsync(const_cast<float *>(P.d_rope), next.rope.data(), next.rope.size() * sizeof(float),
-                            cudaMemcpyHostToDevice, s) != cudaSuccess)
+                            cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(P.d_tbase, &next.rope_tbase, sizeof(int32_t), cudaMemcpyHostToDevice, s) != cudaSuccess)
             return BCA_ERR_CUDA;
     }
     P.videos.swap(next.videos);

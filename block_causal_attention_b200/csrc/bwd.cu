@@ -104,7 +104,7 @@ struct BwdArgs {
     float *dk, *dv, *dkc, *dvc;
     float *dgain_k, *dbase;  // optional parameter gradients (K gain; RoPE bases, shared with Q)
     float coef[24];          // d(base_a^(-k/P))/d(base_a) at [8 a + k]
-    int32_t tbase;           // absolute frame of packed t = 0
+    const int32_t *tbase;    // absolute frame of packed t = 0 (device: rewritten when the window slides)
     int accumulate;          // add dK, dV (and the cache's) into the outputs instead of writing them
     int *status;
 };
@@ -123,7 +123,7 @@ struct DqArgs {
     float *dq;
     float *dgain_q, *dbase;  // optional parameter gradients (Q gain; RoPE bases, shared with K)
     float coef[24];
-    int32_t tbase;
+    const int32_t *tbase;  // absolute frame of packed t = 0 (device)
     int accumulate;  // add dQ into the output instead of writing it
 };
 
@@ -758,7 +758,7 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                     load_row_bf16<D>(a.k + ((size_t)nn * a.hkv + g) * D, x);
                     if (want_pg)
                         qk_param_grads<D>(x, gk, __ldg(a.pos + nn), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps,
-                                          a.coef, a.tbase, pg, pb);
+                                          a.coef, __ldg(a.tbase), pg, pb);
                     qk_prologue_bwd<D>(x, gk, __ldg(a.pos + nn), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps);
                     dst = a.dk + ((size_t)nn * a.hkv + g) * D;
                 }
@@ -820,7 +820,7 @@ __global__ void __launch_bounds__(128) bwd_dq_kernel(DqArgs a) {
         load_row_bf16<D>(a.q + row * D, x);
         if (want_pg)
             qk_param_grads<D>(x, g, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps, a.coef,
-                              a.tbase, pg, pb);
+                              __ldg(a.tbase), pg, pb);
         qk_prologue_bwd<D>(x, g, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps);
         float *dst = a.dq + row * D;
 #pragma unroll
@@ -979,7 +979,7 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     ba.dgain_k = io.dk_gain;
     ba.dbase = io.drope_base;
     for (int i = 0; i < 24; ++i) ba.coef[i] = P.rope_base_coef[i];
-    ba.tbase = P.rope_tbase;
+    ba.tbase = P.d_tbase;
     ba.accumulate = io.accumulate;
     ba.status = P.d_status;
     {
@@ -1007,7 +1007,7 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     da.dgain_q = io.dq_gain;
     da.dbase = io.drope_base;
     for (int i = 0; i < 24; ++i) da.coef[i] = P.rope_base_coef[i];
-    da.tbase = P.rope_tbase;
+    da.tbase = P.d_tbase;
     da.accumulate = io.accumulate;
     {
         ProfScope ps(P, BCA_KERNEL_BWD_DQ, stream);

@@ -296,8 +296,10 @@ int compile_plan(Plan &P) {
 // Packed positions of the new tokens and the RoPE cos/sin tables, from P.videos.  The
 // t field holds t - tbase (tbase = the smallest t0 of a non-empty video) and the t table
 // covers [tbase, tbase + extent), so a window that slides by shifting every t0 keeps
-// the same table size (bca_plan_update_positions relies on that).
-int build_positions(Plan &P) {
+// the same table size.  With `layout` (bca_plan_update_positions on an uploaded plan)
+// the axis offsets and table size are taken from it, and a t or h extent that does not
+// fit returns BCA_ERR_UNSUPPORTED.
+int build_positions(Plan &P, const Plan *layout) {
     P.pos.resize(P.nq);
     int32_t tbase = INT32_MAX;
     for (const bca_video &v : P.videos)
@@ -323,10 +325,21 @@ int build_positions(Plan &P) {
     P.rope_pairs = pairs;
     P.rope_tbase = tbase;
     const int32_t ext[3] = {tmax + 1, hmax + 1, wmax + 1};
-    P.rope_axis_off[0] = 0;
-    P.rope_axis_off[1] = ext[0];
-    P.rope_axis_off[2] = ext[0] + ext[1];
-    P.rope.assign((size_t)(ext[0] + ext[1] + ext[2]) * pairs * 2, 0.0f);
+    if (layout) {
+        // Keep the table layout of an uploaded plan: its launches (also those captured in
+        // CUDA graphs) hold the axis offsets by value, so only the entries may change.
+        const int32_t *lo = layout->rope_axis_off;
+        if (ext[0] > lo[1] || ext[1] > lo[2] - lo[1] ||
+            (size_t)(lo[2] + ext[2]) * pairs * 2 > layout->rope_capacity)
+            return BCA_ERR_UNSUPPORTED;
+        for (int a = 0; a < 3; ++a) P.rope_axis_off[a] = lo[a];
+        P.rope.assign(layout->rope_capacity, 0.0f);
+    } else {
+        P.rope_axis_off[0] = 0;
+        P.rope_axis_off[1] = ext[0];
+        P.rope_axis_off[2] = ext[0] + ext[1];
+        P.rope.assign((size_t)(ext[0] + ext[1] + ext[2]) * pairs * 2, 0.0f);
+    }
     for (int a = 0; a < 3; ++a) {
         for (int32_t pp = 0; pp < ext[a]; ++pp) {
             const double position = (double)pp + (a == 0 ? (double)tbase : 0.0);

@@ -75,6 +75,7 @@ struct Plan {
     const uint32_t *d_pos = nullptr;
     const float *d_rope = nullptr;
     int *d_status = nullptr;
+    int32_t *d_tbase = nullptr;      // rope_tbase on the device (read by the backward's base gradient)
 
     // per-kernel timing (bca_profile_enable); events are CUDA event handles
     struct ProfRecord {
@@ -91,7 +92,7 @@ int validate_problem(const bca_problem *p, Plan &plan);
 int compile_plan(Plan &plan);
 // Positions and RoPE tables from plan.videos (part of compile_plan; also used when only
 // the videos' start frames change).
-int build_positions(Plan &plan);
+int build_positions(Plan &plan, const Plan *layout = nullptr);
 // Expand compiled tiles of rows [r0, r1) into a coverage map (host).
 int expand_rows(const Plan &plan, int64_t r0, int64_t r1, uint8_t *out);
 // Same from the transposed (backward) runs, for keys [k0, k1): out[(j - k0) * nq + i].

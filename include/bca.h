@@ -163,10 +163,13 @@ int bca_plan_expand_cols(bca_plan_t plan, int64_t key_begin, int64_t key_end, ui
  * work items are unchanged and only the new tokens' positions and RoPE tables are
  * rewritten (cudaMemcpyAsync on `stream`, after any launch already queued there; the
  * host arguments may be freed on return).  Tables are stored relative to the smallest t0,
- * so shifting every t0 by the same amount keeps their size; a change that would enlarge
- * the t range returns BCA_ERR_UNSUPPORTED and changes nothing.  Launches captured in a
- * CUDA graph keep working: they read the rewritten tables in place.  Returns
- * BCA_ERR_INVALID_ARGUMENT for a changed geometry or a negative t0. */
+ * so shifting every t0 by the same amount keeps their size.  The table layout (where the
+ * t, h and w sections start, and its size) is fixed when the plan is created: videos may
+ * move by different amounts as long as the span of frames they cover is not longer than
+ * the plan's first one; a longer span returns BCA_ERR_UNSUPPORTED and changes nothing.
+ * Launches captured in a CUDA graph keep working: they read the rewritten positions,
+ * tables and first frame (used by the RoPE-base gradient of bca_bwd_ex) in place.
+ * Returns BCA_ERR_INVALID_ARGUMENT for a changed geometry or a negative t0. */
 int bca_plan_update_positions(bca_plan_t plan, const bca_video *videos, int num_videos, void *stream);
 
 /* Bytes of caller-provided device workspace a pass needs (16-byte aligned).  The
@@ -195,8 +198,15 @@ int bca_fwd(bca_plan_t plan, const void *q, const void *k, const void *v,
  *  - Limit: problems whose bca_workspace_bytes(plan, BCA_PASS_FWD) exceeds
  *    BCA_STATIC_WORKSPACE_BYTES are rejected with BCA_ERR_TOO_LARGE, before any
  *    launch.  (16 MiB holds, e.g., 6144 keys x 8 KV heads at head_dim 48.)
+ *  - The array occupies BCA_STATIC_WORKSPACE_BYTES on every GPU on which the library's
+ *    module is loaded, whether or not this entry point is ever called.
+ *  - The plan must belong to the current device (the one it was created on), else the
+ *    call returns BCA_ERR_INVALID_ARGUMENT.
  *  - The first call on a device looks up the array's device address once (with
  *    that device current); make that first call before any stream capture begins.
+ *    The address is kept for the life of the process: after a cudaDeviceReset (or any
+ *    other teardown of the device's primary context) it is stale, so do not call this
+ *    entry point again in that process after such a reset.
  *  - Every call on a device shares the one array and leaves its contents behind.
  *    Each call rewrites every byte it reads before reading it, so nothing needs to
  *    start at zero, but calls whose kernels overlap on the GPU (other streams, or
