@@ -267,18 +267,29 @@ def seeded_normal_bf16(seed: int, shape: Sequence[int], device="cpu",
     return out.view((nrows,) + shape[1:])
 
 
-def seeded_rows_bf16(seed: int, shape: Sequence[int], rows, device="cpu") -> torch.Tensor:
-    """Selected rows (any order) of the same seeded tensor."""
+def seeded_rows_bf16(seed: int, shape: Sequence[int], rows, device="cpu", heads=None) -> torch.Tensor:
+    """Selected rows (any order) of the same seeded tensor; with ``heads`` = (h0, h1) only
+    heads [h0, h1) of a [rows, heads, D] tensor (the same elements as the full rows')."""
     shape = tuple(int(s) for s in shape)
     row_elems = int(np.prod(shape[1:]))
+    cols = torch.arange(row_elems, device=device)
+    out_shape = shape[1:]
+    if heads is not None:
+        h0, h1 = int(heads[0]), int(heads[1])
+        cols = cols[h0 * shape[2]:h1 * shape[2]]
+        out_shape = (h1 - h0,) + shape[2:]
     rows = torch.as_tensor(np.asarray(rows, dtype=np.int64), device=device)
-    e = (rows[:, None] * row_elems + torch.arange(row_elems, device=device)[None, :]).reshape(-1)
-    lo = e & _M32
-    hi = e >> 32
-    key = _mix32(((hi + 1) * _SEED_MUL + seed) & _M32)
-    h = _mix32(lo ^ key)
-    h = _mix32((h + seed * 0x9E37) & _M32)
-    return _quantile_table(device)[h >> 16].view((len(rows),) + shape[1:])
+    out = torch.empty((len(rows), len(cols)), dtype=torch.bfloat16, device=device)
+    step = max(1, (1 << 24) // max(1, len(cols)))
+    for r0 in range(0, len(rows), step):
+        e = (rows[r0:r0 + step, None] * row_elems + cols[None, :]).reshape(-1)
+        lo = e & _M32
+        hi = e >> 32
+        key = _mix32(((hi + 1) * _SEED_MUL + seed) & _M32)
+        h = _mix32(lo ^ key)
+        h = _mix32((h + seed * 0x9E37) & _M32)
+        out[r0:r0 + step] = _quantile_table(device)[h >> 16].view(-1, len(cols))
+    return out.view((len(rows),) + tuple(out_shape))
 
 
 def tensor_shape(w: Workload, tid: int) -> tuple:
@@ -299,8 +310,8 @@ def make_input(w: Workload, tid: int, device="cpu", row_start=0, nrows=None) -> 
     return seeded_normal_bf16(seed_of(w, tid), tensor_shape(w, tid), device, row_start, nrows)
 
 
-def make_input_rows(w: Workload, tid: int, rows, device="cpu") -> torch.Tensor:
-    return seeded_rows_bf16(seed_of(w, tid), tensor_shape(w, tid), rows, device)
+def make_input_rows(w: Workload, tid: int, rows, device="cpu", heads=None) -> torch.Tensor:
+    return seeded_rows_bf16(seed_of(w, tid), tensor_shape(w, tid), rows, device, heads)
 
 
 def make_inputs(w: Workload, device="cpu", with_grad: bool = False) -> dict:

@@ -413,3 +413,70 @@ def test_video_key_grads_equal_the_dense_backward():
             k_dk, k_dv = video_key_grads(w, vi, g, keys)
             assert np.abs(k_dk - dk[start + keys, g]).max() <= 1e-12
             assert np.abs(k_dv - dv[start + keys, g]).max() <= 1e-12
+
+
+# --------------------------------------------------------------------------- full-size helpers
+
+def test_blas_rows_equal_the_loop_rows_on_random_slice_unions():
+    """attn_fwd_rows_blas (fp64 matrix products over row batches) gives the per-pair C
+    loops' O and LSE on random FULL/CAUSAL slice unions with empty rows, GQA and MHA,
+    rows in any order and batches that split the rows raggedly."""
+    rng = np.random.default_rng(77)
+    for trial in range(6):
+        nq, nc = int(rng.integers(20, 90)), int(rng.integers(0, 40))
+        nk = nq + nc
+        Hq, Hkv = ((8, 2), (4, 4), (6, 1))[trial % 3]
+        D = (24, 32, 48)[trial % 3]
+        sl = []
+        for _ in range(int(rng.integers(1, 5))):
+            q0 = int(rng.integers(0, nq)); q1 = int(rng.integers(q0, nq + 1))
+            k0 = int(rng.integers(0, nk)); k1 = int(rng.integers(k0, nk + 1))
+            sl.append((q0, q1, k0, k1, int(rng.integers(0, 2))))
+        sl = np.asarray(sl, np.int64)
+        qh, kh, v = _rand((nq, Hq, D)), _rand((nk, Hkv, D)), _rand((nk, Hkv, D))
+        rows = rng.permutation(nq)[:int(rng.integers(1, nq + 1))]
+        O1, l1 = oracle.attn_fwd_rows(qh[rows], rows, kh, v, sl, Hq, Hkv)
+        O2, l2 = oracle.attn_fwd_rows_blas(qh[rows], rows, kh, v, sl, Hq, Hkv, batch=7, workers=3)
+        assert np.array_equal(np.isneginf(l1), np.isneginf(l2))
+        fin = np.isfinite(l1)
+        assert np.abs(l1[fin] - l2[fin]).max(initial=0) <= 1e-12
+        assert np.abs(O1 - O2).max() <= 1e-12
+
+
+def test_blas_rows_one_chunk_equals_full_attention():
+    n, Hq, Hkv, D = 45, 8, 2, 48
+    qh, kh, v = _rand((n, Hq, D)), _rand((n, Hkv, D)), _rand((n, Hkv, D))
+    O, lse = oracle.attn_fwd_rows_blas(qh, np.arange(n), kh, v, _block_causal([1], n), Hq, Hkv, batch=8)
+    assert np.allclose(O, _sdpa(qh, kh, v), atol=1e-12)
+    s = (qh[7, 5] @ kh[:, 1].T) / math.sqrt(D)   # head 5 of 8 over 2 KV heads uses KV head 1
+    assert abs(lse[7, 5] - (s.max() + math.log(np.exp(s - s.max()).sum()))) < 1e-12
+
+
+@pytest.mark.parametrize("name", ["kvrange_replica", "packed_replica", "cache_small"])
+def test_golden_key_grads_script_equals_the_dense_backward(name):
+    """The script that writes the full-size dK / dV expectations (tests/golden/
+    make_key_grads.py: rows that see the sampled keys only, forward by row batches, key
+    backward) gives the dense oracle backward's dK, dV and cache gradients on small
+    workloads of the same structure (KV-range transitions, packed videos, a KV cache)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("make_key_grads", os.path.join(GOLDEN, "make_key_grads.py"))
+    mk = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mk)
+    if name == "cache_small":
+        w = W._c3_like("cache_small", 98, 1, 5, 5, 4, 1, backward=True)    # 8 cached + 4 new chunks of 25
+    else:
+        w = W.WORKLOADS[name]
+    x = W.make_inputs(w, "cpu", with_grad=True)
+    _, dk, dv, dkc, dvc, _, _ = oracle.backward(x["q"], x["k"], x["v"], x["k_cache"], x["v_cache"], x["do"],
+                                                w.videos_array(), w.slices_array(), w.hq, w.hkv,
+                                                base=w.rope_base, eps=w.eps)
+    rng = np.random.default_rng(5)
+    keys = np.unique(np.concatenate([[0, w.nk - 1], rng.integers(0, w.nk, 40)]))
+    nc = w.num_cache_keys
+    for g in sorted({0, w.hkv - 1}):
+        k_dk, k_dv, _ = mk.key_grads(w, g, keys, workers=2)
+        for a, j in enumerate(keys):
+            want_k = dkc[j, g] if j < nc else dk[j - nc, g]
+            want_v = dvc[j, g] if j < nc else dv[j - nc, g]
+            assert np.abs(k_dk[a] - want_k).max() <= 1e-12, (g, j)
+            assert np.abs(k_dv[a] - want_v).max() <= 1e-12, (g, j)
