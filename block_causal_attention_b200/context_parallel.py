@@ -295,6 +295,13 @@ def _default_engine(hq, hkv, d, videos, num_cache_keys, slices, rope_base, eps, 
     return Plan(hq, hkv, d, videos, num_cache_keys, slices, rope_base, eps, o_fp32)
 
 
+def _host_staged(group, t) -> bool:
+    """True when the collectives of `group` cannot take `t` where it lives: device tensors
+    on a gloo group (gloo moves host memory), which are then exchanged through host copies."""
+    import torch.distributed as dist
+    return t.is_cuda and dist.get_backend(group) == "gloo"
+
+
 def _all_to_all_rows(group, send: List, recv_counts: List[int], row_shape, like, async_op: bool = False):
     """Rows of `send[dst]` go to rank dst; returns the received rows per source rank (and,
     with async_op, the pending work to wait on before reading them).  Rows are moved
@@ -312,6 +319,11 @@ def _all_to_all_rows(group, send: List, recv_counts: List[int], row_shape, like,
     work = None
     if world == 1:
         rview.copy_(sview)
+    elif _host_staged(group, sview):
+        rhost = torch.empty(rview.shape, dtype=rview.dtype)
+        dist.all_to_all_single(rhost, sview.cpu(), output_split_sizes=list(recv_counts),
+                               input_split_sizes=[int(f.shape[0]) for f in flat], group=group)
+        rview.copy_(rhost)
     else:
         work = dist.all_to_all_single(rview, sview, output_split_sizes=list(recv_counts),
                                       input_split_sizes=[int(f.shape[0]) for f in flat], group=group,
@@ -423,8 +435,13 @@ class ContextParallelAttention:
             gk.index_add_(0, rows, dkc[:ncl])
             gv.index_add_(0, rows, dvc[:ncl])
         if self.world > 1:
-            dist.all_reduce(gk, group=self.group)
-            dist.all_reduce(gv, group=self.group)
+            for t in (gk, gv):
+                if _host_staged(self.group, t):
+                    h = t.cpu()
+                    dist.all_reduce(h, group=self.group)
+                    t.copy_(h)
+                else:
+                    dist.all_reduce(t, group=self.group)
         return gk, gv
 
     def _return_grads_start(self, rem_k, rem_v):
