@@ -26,10 +26,16 @@ class Plan:
 
     def __init__(self, hq: int, hkv: int, d: int, videos, num_cache_keys: int = 0, slices=None,
                  rope_base=(1e4, 1e4, 1e4), eps: float = 1e-6, o_fp32: bool = False,
-                 host_only: bool = False, test_force_timeout: bool = False, fp8: bool = False):
-        """fp8=True: forward with e4m3 tensor-core operands (BCA_FWD_FP8_E4M3; forward only)."""
+                 host_only: bool = False, test_force_timeout: bool = False, fp8: bool = False,
+                 no_prologue: bool = False, dq_deterministic: bool = False, cache_k_fp16: bool = False):
+        """fp8=True: forward with e4m3 tensor-core operands (BCA_FWD_FP8_E4M3; forward only).
+        no_prologue=True: q and k are given post-prologue (BCA_NO_PROLOGUE).
+        dq_deterministic=True: dQ by a separate fixed-order pass (BCA_DQ_DETERMINISTIC).
+        cache_k_fp16=True: k_cache is fp16 and k_prologue writes fp16 (BCA_CACHE_K_FP16)."""
         flags = (_abi.BCA_O_FP32 if o_fp32 else 0) | (_abi.BCA_PLAN_HOST_ONLY if host_only else 0) | \
-            (_abi.BCA_TEST_FORCE_TIMEOUT if test_force_timeout else 0) | (_abi.BCA_FWD_FP8_E4M3 if fp8 else 0)
+            (_abi.BCA_TEST_FORCE_TIMEOUT if test_force_timeout else 0) | (_abi.BCA_FWD_FP8_E4M3 if fp8 else 0) | \
+            (_abi.BCA_NO_PROLOGUE if no_prologue else 0) | (_abi.BCA_DQ_DETERMINISTIC if dq_deterministic else 0) | \
+            (_abi.BCA_CACHE_K_FP16 if cache_k_fp16 else 0)
         prob, keep = _abi.make_problem(hq, hkv, d, videos, num_cache_keys, slices, rope_base, eps, flags)
         self._lib = _abi.lib()
         self._h = _abi.ctypes.c_void_p()
@@ -39,6 +45,7 @@ class Plan:
         self.hq, self.hkv, self.d = int(hq), int(hkv), int(d)
         self.o_fp32 = bool(o_fp32)
         self.fp8 = bool(fp8)
+        self.cache_k_fp16 = bool(cache_k_fp16)
         self.host_only = bool(host_only)
         self.num_cache_keys = int(num_cache_keys)
         inf = self.info()
@@ -109,10 +116,11 @@ class Plan:
                 raise ValueError(f"{name}: expected contiguous bf16 CUDA tensor of shape "
                                  f"{(rows, heads, self.d)}, got {t.dtype} {tuple(t.shape)}")
         if self.num_cache_keys:
-            for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
-                if t is None or t.dtype != torch.bfloat16 or not t.is_contiguous() or \
+            kdt = torch.float16 if self.cache_k_fp16 else torch.bfloat16
+            for name, t, dt in (("k_cache", k_cache, kdt), ("v_cache", v_cache, torch.bfloat16)):
+                if t is None or t.dtype != dt or not t.is_contiguous() or \
                         tuple(t.shape) != (self.num_cache_keys, self.hkv, self.d):
-                    raise ValueError(f"{name}: expected bf16 [{self.num_cache_keys}, {self.hkv}, {self.d}]")
+                    raise ValueError(f"{name}: expected {dt} [{self.num_cache_keys}, {self.hkv}, {self.d}]")
         dev = q.device
         if o is None:
             o = torch.empty((self.nq, self.hq, self.d), device=dev,
@@ -189,7 +197,8 @@ class Plan:
         """Post-prologue keys (bf16 [Nq, Hkv, D]) of the plan's new tokens."""
         import torch
         if out is None:
-            out = torch.empty((self.nq, self.hkv, self.d), device=k.device, dtype=torch.bfloat16)
+            out = torch.empty((self.nq, self.hkv, self.d), device=k.device,
+                              dtype=torch.float16 if self.cache_k_fp16 else torch.bfloat16)
         _abi.check(self._lib.bca_k_prologue(self._h, _ptr(k), _ptr(k_gain), _ptr(out), self._stream(stream)),
                    "bca_k_prologue")
         return out

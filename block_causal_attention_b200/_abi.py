@@ -29,6 +29,9 @@ BCA_O_FP32 = 0x1
 BCA_PLAN_HOST_ONLY = 0x2
 BCA_TEST_FORCE_TIMEOUT = 0x4
 BCA_FWD_FP8_E4M3 = 0x8
+BCA_NO_PROLOGUE = 0x10
+BCA_DQ_DETERMINISTIC = 0x20
+BCA_CACHE_K_FP16 = 0x40
 BCA_PASS_FWD = 0
 BCA_PASS_BWD = 1
 
@@ -42,7 +45,7 @@ EXPORTS = ("bca_plan_create", "bca_plan_destroy", "bca_plan_get_info", "bca_plan
 BCA_KERNEL_KV_IMAGE = 0
 BCA_KERNEL_FWD = 1
 KERNEL_NAMES = {0: "kv_image_kernel", 1: "fwd_kernel", 2: "bwd_prep_kernel", 3: "bwd_kv_image_kernel",
-                4: "bwd_kernel", 5: "bwd_dq_kernel"}
+                4: "bwd_kernel", 5: "bwd_dq_kernel", 6: "bwd_dq_pass_kernel"}
 
 
 class bca_slice(ctypes.Structure):

@@ -239,6 +239,7 @@ int bca_fwd(bca_plan_t plan, const void *q, const void *k, const void *v, const 
     if (P.nq == 0) return BCA_OK;
     if (!q || !k || !v || !o || !lse || !workspace) return BCA_ERR_INVALID_ARGUMENT;
     if (P.nc > 0 && (!k_cache || !v_cache)) return BCA_ERR_INVALID_ARGUMENT;
+    if ((P.flags & BCA_NO_PROLOGUE) && (q_gain || k_gain)) return BCA_ERR_INVALID_ARGUMENT;
     const void *ptrs[] = {q, k, v, k_cache, v_cache, q_gain, k_gain, o, lse, workspace};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return BCA_ERR_MISALIGNED;
@@ -267,6 +268,8 @@ int bca_bwd_ex(bca_plan_t plan, const void *q, const void *k, const void *v, con
         return BCA_OK;
     }
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return BCA_ERR_INVALID_ARGUMENT;
+    if ((P.flags & BCA_NO_PROLOGUE) && (q_gain || k_gain || dq_gain || dk_gain || drope_base))
+        return BCA_ERR_INVALID_ARGUMENT;
     if (P.nc > 0 && (!k_cache || !v_cache)) return BCA_ERR_INVALID_ARGUMENT;
     const void *ptrs[] = {q, k, v, k_cache, v_cache, q_gain, k_gain, o, lse, dout, dq, dk, dv, dk_cache, dv_cache,
                           workspace};
@@ -310,6 +313,7 @@ int bca_k_prologue(bca_plan_t plan, const void *k, const float *k_gain, void *k_
     if (rc != BCA_OK) return rc;
     if (P.nq == 0) return BCA_OK;
     if (!k || !k_hat) return BCA_ERR_INVALID_ARGUMENT;
+    if ((P.flags & BCA_NO_PROLOGUE) && k_gain) return BCA_ERR_INVALID_ARGUMENT;
     if (!aligned16(k) || !aligned16(k_hat) || (k_gain && !aligned16(k_gain))) return BCA_ERR_MISALIGNED;
     return bca::launch_k_prologue(P, k, k_gain, k_hat, static_cast<cudaStream_t>(stream));
 }
@@ -322,6 +326,7 @@ int bca_k_prologue_bwd(bca_plan_t plan, const void *k, const float *k_gain, cons
     if (rc != BCA_OK) return rc;
     if (P.nq == 0) return BCA_OK;
     if (!k || !dk_hat || !dk) return BCA_ERR_INVALID_ARGUMENT;
+    if ((P.flags & BCA_NO_PROLOGUE) && k_gain) return BCA_ERR_INVALID_ARGUMENT;
     if (!aligned16(k) || !aligned16(dk_hat) || !aligned16(dk) || (k_gain && !aligned16(k_gain)))
         return BCA_ERR_MISALIGNED;
     return bca::launch_k_prologue_bwd(P, k, k_gain, dk_hat, dk, accumulate, static_cast<cudaStream_t>(stream));

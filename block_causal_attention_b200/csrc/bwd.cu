@@ -63,6 +63,7 @@ struct PrepArgs {
     int64_t nq, nqt;
     int hq;
     float eps, qscale;
+    int prologue;  // 0: rows given post-prologue (BCA_NO_PROLOGUE)
     __half *qimg16;
     __nv_bfloat16 *doimg;
     float *lse2, *dsum;
@@ -78,6 +79,8 @@ struct BwdKVArgs {
     int64_t nc, nk, nkt;
     int hkv;
     float eps;
+    int prologue;
+    int kc_f16;  // cache keys are fp16 (BCA_CACHE_K_FP16)
     __half *kimg16;
     __nv_bfloat16 *vimg;
     float *bounds;  // [1] = max |v_j|
@@ -100,6 +103,7 @@ struct BwdArgs {
     int64_t nq, nk, nc, nqt, nkt;
     int hq, hkv;
     float eps;
+    int prologue;
     float *dqacc;  // fp32 dQ-hat accumulator, [Hq][query tile][2][128][DPAD / 2]
     float *dk, *dv, *dkc, *dvc;
     float *dgain_k, *dbase;  // optional parameter gradients (K gain; RoPE bases, shared with Q)
@@ -107,6 +111,9 @@ struct BwdArgs {
     const int32_t *tbase;    // absolute frame of packed t = 0 (device: rewritten when the window slides)
     int accumulate;          // add dK, dV (and the cache's) into the outputs instead of writing them
     int *status;
+    uint64_t timeout_ns;     // per wait
+    int skip_loads;          // failure-detection test: issue no loads, so every wait runs out
+    int dq_pass;             // 1: dQ comes from bwd_dq_pass_kernel (BCA_DQ_DETERMINISTIC), not from here
 };
 
 struct DqArgs {
@@ -118,6 +125,7 @@ struct DqArgs {
     int64_t nq, nqt;
     int hq;
     float eps, scale;
+    int prologue;
     const float *bounds;
     const float *dqacc;
     float *dq;
@@ -191,7 +199,8 @@ __global__ void __launch_bounds__(128) bwd_prep_kernel(PrepArgs a) {
     float x[D];
     if (live) {
         load_row_bf16<D>(a.q + row, x);
-        qk_prologue<D>(x, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps, a.qscale);
+        qk_prologue<D>(x, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps, a.qscale,
+                       a.prologue != 0);
     } else {
 #pragma unroll
         for (int d = 0; d < D; ++d) x[d] = 0.f;
@@ -245,11 +254,12 @@ __global__ void __launch_bounds__(128) bwd_kv_image_kernel(BwdKVArgs a) {
     const size_t tile = ((size_t)g * a.nkt + kt) * (128 * DPAD);
     float x[D];
     if (key < a.nc) {
-        load_row_bf16<D>(a.kc + ((size_t)key * a.hkv + g) * D, x);
+        load_row_16<D>(a.kc + ((size_t)key * a.hkv + g) * D, a.kc_f16 != 0, x);
     } else if (key < a.nk) {
         const int64_t n = key - a.nc;
         load_row_bf16<D>(a.k + ((size_t)n * a.hkv + g) * D, x);
-        qk_prologue<D>(x, __ldg(a.pos + n), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps, 1.0f);
+        qk_prologue<D>(x, __ldg(a.pos + n), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps, 1.0f,
+                       a.prologue != 0);
     } else {
 #pragma unroll
         for (int d = 0; d < D; ++d) x[d] = 0.f;
@@ -362,20 +372,21 @@ struct ItemCursor {
     }
 };
 
-__device__ __forceinline__ bool wait_abort(uint32_t bar, uint32_t parity, int *status, volatile int *abort_flag) {
+__device__ __forceinline__ bool wait_abort(uint32_t bar, uint32_t parity, int *status, volatile int *abort_flag,
+                                           uint64_t timeout_ns) {
     // A completed phase needs no look at the abort flag (a volatile shared load on every
     // waiter's path); only a wait that would block has to know whether the CTA gives up.
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (mbar_wait(bar, parity, kWaitTimeoutNs)) return true;
+    if (mbar_wait(bar, parity, timeout_ns)) return true;
     atomicOr(status, kStatusTimeout);
     *abort_flag = 1;
     return false;
 }
 
 __device__ __forceinline__ bool warp_wait_abort(uint32_t bar, uint32_t parity, int *status,
-                                                volatile int *abort_flag) {
-    const bool ok = wait_abort(bar, parity, status, abort_flag);
+                                                volatile int *abort_flag, uint64_t timeout_ns) {
+    const bool ok = wait_abort(bar, parity, status, abort_flag, timeout_ns);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -437,7 +448,7 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
 
     if (warp == 0) {
         // ------------------------------------------------ producer
-        if (lane == 0) {
+        if (lane == 0 && !a.skip_loads) {
             const size_t ktile = ((size_t)g * a.nkt + kt) * (128 * DPAD);
             mbar_arrive_expect_tx(bar(L::B_KV), 2 * L::TILE);
             bulk_g2s(sbase + L::OFF_K16, a.kimg16 + ktile, L::TILE, bar(L::B_KV));
@@ -447,7 +458,7 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
             for (int i = 0; i < n; ++i, cur.next()) {
                 const int s = i % STAGES;
                 if (i >= STAGES &&
-                    !wait_abort(bar(L::B_ST_EMPTY + s), ((i / STAGES) - 1) & 1, a.status, abort_flag))
+                    !wait_abort(bar(L::B_ST_EMPTY + s), ((i / STAGES) - 1) & 1, a.status, abort_flag, a.timeout_ns))
                     break;
                 const int h = g * G + cur.hh;
                 const size_t qtile = ((size_t)h * a.nqt + cur.qt) * (128 * DPAD);
@@ -465,9 +476,9 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
             // every issued copy must have landed before the CTA may exit (matters when
             // the consumers stopped early)
             for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
-                if (!mbar_wait(bar(L::B_ST_FULL + j % STAGES), (j / STAGES) & 1, kWaitTimeoutNs))
+                if (!mbar_wait(bar(L::B_ST_FULL + j % STAGES), (j / STAGES) & 1, a.timeout_ns))
                     atomicOr(a.status, kStatusTimeout);
-            if (!mbar_wait(bar(L::B_KV), 0, kWaitTimeoutNs)) atomicOr(a.status, kStatusTimeout);
+            if (!mbar_wait(bar(L::B_KV), 0, a.timeout_ns)) atomicOr(a.status, kStatusTimeout);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -521,8 +532,8 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                     mma_f16(tbase + L::COL_DQ, dds_mn + bo + (uint64_t)(kk * 16), dkmn + (uint64_t)(kk * 16), IDESC_DQ,
                             kk > 0);
             };
-            bool ok = wait_abort(bar(L::B_KV), 0, a.status, abort_flag);
-            if (ok && n > 0) ok = wait_abort(bar(L::B_ST_FULL), 0, a.status, abort_flag);
+            bool ok = wait_abort(bar(L::B_KV), 0, a.status, abort_flag, a.timeout_ns);
+            if (ok && n > 0) ok = wait_abort(bar(L::B_ST_FULL), 0, a.status, abort_flag, a.timeout_ns);
             tc_fence_after();
             if (ok && n > 0) {
                 issue_s_dp(0);
@@ -531,32 +542,34 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
             for (int i = 0; i < n && ok; ++i) {
                 if (i + 1 < n) {
                     ok = wait_abort(bar(L::B_ST_FULL + (i + 1) % STAGES), ((i + 1) / STAGES) & 1, a.status,
-                                    abort_flag) &&
-                         wait_abort(bar(L::B_S_FREE), i & 1, a.status, abort_flag);
+                                    abort_flag, a.timeout_ns) &&
+                         wait_abort(bar(L::B_S_FREE), i & 1, a.status, abort_flag, a.timeout_ns);
                     if (!ok) break;
                     tc_fence_after();
                     issue_s_dp(i + 1);
                     mma_commit(bar(L::B_S_FULL));
                 }
                 const int b = i & 1;
-                ok = wait_abort(bar(L::B_DS_READY), i & 1, a.status, abort_flag);
+                ok = wait_abort(bar(L::B_DS_READY), i & 1, a.status, abort_flag, a.timeout_ns);
                 if (!ok) break;
                 tc_fence_after();
                 issue_dv(i);
                 mma_commit(bar(L::B_PT_FREE));
                 issue_dk(i);
                 mma_commit(bar(L::B_ST_EMPTY + i % STAGES));
-                if (i > 0) {  // the compute warps have read dQ_part of item i - 1
-                    ok = wait_abort(bar(L::B_DQ_FREE), (i - 1) & 1, a.status, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
+                if (!a.dq_pass) {
+                    if (i > 0) {  // the compute warps have read dQ_part of item i - 1
+                        ok = wait_abort(bar(L::B_DQ_FREE), (i - 1) & 1, a.status, abort_flag, a.timeout_ns);
+                        if (!ok) break;
+                        tc_fence_after();
+                    }
+                    issue_dq(i);
+                    mma_commit(bar(L::B_DQ_FULL));
                 }
-                issue_dq(i);
-                mma_commit(bar(L::B_DQ_FULL));
                 mma_commit(bar(L::B_DS_FREE + b));
             }
             mma_commit(bar(L::B_MMA_DONE));
-            if (!mbar_wait(bar(L::B_MMA_DONE), 0, kWaitTimeoutNs)) {
+            if (!mbar_wait(bar(L::B_MMA_DONE), 0, a.timeout_ns)) {
                 atomicOr(a.status, kStatusTimeout);
                 *abort_flag = 1;
             }
@@ -580,7 +593,7 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
         // reduce (TMA engine); the tile of (head, query tile) is laid out
         // [2 column halves][128 rows][HALF], so the block is contiguous
         auto dq_epilogue = [&](int j, int qt_j, int h_j) -> bool {
-            if (!warp_wait_abort(bar(L::B_DQ_FULL), j & 1, a.status, abort_flag)) return false;
+            if (!warp_wait_abort(bar(L::B_DQ_FULL), j & 1, a.status, abort_flag, a.timeout_ns)) return false;
             tc_fence_after();
             uint32_t v[HALF];
 #pragma unroll
@@ -611,8 +624,8 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
             const int s = i % STAGES;
             const int h = g * G + cur.hh;
             const uint8_t *st = smem + L::OFF_STAGE + s * L::STAGE_BYTES;
-            ok = warp_wait_abort(bar(L::B_ST_FULL + s), (i / STAGES) & 1, a.status, abort_flag) &&
-                 warp_wait_abort(bar(L::B_S_FULL), i & 1, a.status, abort_flag);
+            ok = warp_wait_abort(bar(L::B_ST_FULL + s), (i / STAGES) & 1, a.status, abort_flag, a.timeout_ns) &&
+                 warp_wait_abort(bar(L::B_S_FULL), i & 1, a.status, abort_flag, a.timeout_ns);
             if (!ok) break;
             tc_fence_after();
             // S^T / dP^T leave tensor memory 16 columns at a time, the next chunk in flight
@@ -629,10 +642,10 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
             const uint32_t *mask = reinterpret_cast<const uint32_t *>(st + L::ST_MASK);
             const int b = i & 1;
             if (i > 1) {  // dS^T buffer b was last read by the dK / dQ MMAs of item i - 2
-                ok = warp_wait_abort(bar(L::B_DS_FREE + b), ((i >> 1) - 1) & 1, a.status, abort_flag);
+                ok = warp_wait_abort(bar(L::B_DS_FREE + b), ((i >> 1) - 1) & 1, a.status, abort_flag, a.timeout_ns);
             }
             if (ok && i > 0) {  // the dV MMAs of item i - 1 have read P^T from tensor memory
-                ok = warp_wait_abort(bar(L::B_PT_FREE), (i - 1) & 1, a.status, abort_flag);
+                ok = warp_wait_abort(bar(L::B_PT_FREE), (i - 1) & 1, a.status, abort_flag, a.timeout_ns);
                 tc_fence_after();
             }
             if (!ok) {
@@ -700,19 +713,19 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(bar(L::B_DS_READY));
-            if (i > 0 && !dq_epilogue(i - 1, prev_qt, prev_h)) {
+            if (i > 0 && !a.dq_pass && !dq_epilogue(i - 1, prev_qt, prev_h)) {
                 ok = false;
                 break;
             }
             prev_qt = cur.qt;
             prev_h = h;
         }
-        if (ok && n > 0) ok = dq_epilogue(n - 1, prev_qt, prev_h);
+        if (ok && n > 0 && !a.dq_pass) ok = dq_epilogue(n - 1, prev_qt, prev_h);
         if (lane == 0) bulk_wait_group0();  // the reduces have landed and read their staging
 
         // dK / dV epilogue: warpgroup 0 writes dV, warpgroup 1 dK (through the
         // prologue backward for new keys)
-        if (ok && n > 0) ok = warp_wait_abort(bar(L::B_MMA_DONE), 0, a.status, abort_flag);
+        if (ok && n > 0) ok = warp_wait_abort(bar(L::B_MMA_DONE), 0, a.status, abort_flag, a.timeout_ns);
         tc_fence_after();
         float acc[DPAD];
 #pragma unroll
@@ -759,7 +772,8 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
                     if (want_pg)
                         qk_param_grads<D>(x, gk, __ldg(a.pos + nn), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps,
                                           a.coef, __ldg(a.tbase), pg, pb);
-                    qk_prologue_bwd<D>(x, gk, __ldg(a.pos + nn), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps);
+                    qk_prologue_bwd<D>(x, gk, __ldg(a.pos + nn), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps,
+                                       a.prologue != 0);
                     dst = a.dk + ((size_t)nn * a.hkv + g) * D;
                 }
                 if (dst) {
@@ -771,6 +785,291 @@ __global__ void __launch_bounds__(384, 1) bwd_kernel(BwdArgs a) {
             }
         }
         if (want_pg) warp_param_grads_add<D>(pg, pb, a.dgain_k, a.dbase);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tbase, L::TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ deterministic dQ pass
+
+// Plans created with BCA_DQ_DETERMINISTIC: dQ-hat is not summed across key-tile CTAs with
+// reduce-adds (whose order varies between runs) but formed by one CTA per (query tile,
+// query head) that walks the query tile's key tiles in a fixed order, recomputing S and
+// dP (two more products per tile than the key-tile kernel's share of the work):
+//   S = Q-hat K-hat^T, dP = dO V^T      (M = 128 queries, N = 128 keys, K = DPAD)
+//   P sc = exp2(S - LSE2 + log2 sc), dS sc = P sc (dP - Dsum)   (the compute warps)
+//   dQ-hat sc += dS sc K-hat           (M = 128 queries, N = DPAD, K = 128 keys)
+// and writes dQ-hat sc into the accumulator layout that bwd_dq_kernel reads.
+// Roles: warp 0 loads the Q-hat / dO tiles once and streams K-hat / V tiles through a
+// ring; warp 1 (one thread) issues the MMAs; warps 4-11 each take 32 query rows (their
+// TMEM lane quarter) and one half of the 128 key columns.
+template <int D>
+struct DqSmem {
+    static constexpr int DPAD = Geo<D>::DPAD;
+    static constexpr int TILE = 128 * DPAD * 2;
+    static constexpr int STAGES = 4;
+    static constexpr int OFF_Q = 0, OFF_DO = TILE;
+    static constexpr int OFF_K = 2 * TILE;
+    static constexpr int OFF_V = OFF_K + STAGES * TILE;
+    static constexpr int OFF_DS = OFF_V + STAGES * TILE;  // [2] fp16 128 x 128, K-major A operand
+    static constexpr int OFF_BAR = OFF_DS + 2 * 32768;
+    static constexpr int B_QD = 0, B_KV_FULL = 1, B_KV_EMPTY = 1 + STAGES, B_S_FULL = 1 + 2 * STAGES,
+                         B_S_FREE = B_S_FULL + 1, B_DS_READY = B_S_FULL + 2, B_DS_FREE = B_S_FULL + 3 /* [2] */,
+                         B_MMA_DONE = B_S_FULL + 5, NBAR = B_S_FULL + 6;
+    static constexpr int OFF_TMEM_PTR = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_ABORT = OFF_TMEM_PTR + 4;
+    static constexpr int BYTES = OFF_ABORT + 12;
+    static_assert(BYTES <= 232448, "shared memory");
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 256;
+};
+
+struct DqPassArgs {
+    const __half *kimg16, *qimg16;
+    const __nv_bfloat16 *vimg, *doimg;
+    const float *lse2, *dsum;
+    const Item *items;
+    const int32_t *run_off;
+    const Run *runs;
+    const uint32_t *masks;
+    int64_t nqt, nkt;
+    int hq, hkv, heads_per_item;
+    float *dqacc;
+    int *status;
+    uint64_t timeout_ns;
+};
+
+template <int D>
+__global__ void __launch_bounds__(384, 1) bwd_dq_pass_kernel(DqPassArgs a) {
+    using L = DqSmem<D>;
+    constexpr int DPAD = L::DPAD;
+    constexpr int HALF = DPAD / 2;
+    constexpr int STAGES = L::STAGES;
+    constexpr uint32_t IDESC_S = idesc_f32acc(128, 128, kFmtF16);                     // Q-hat K-hat^T
+    constexpr uint32_t IDESC_DP = idesc_f32acc(128, 128, kFmtBF16);                   // dO V^T
+    constexpr uint32_t IDESC_DQ = idesc_f32acc_major(128, DPAD, kFmtF16, 0, 1);       // dS K-hat, B MN-major
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t sbase = smem_u32(smem);
+    auto bar = [&](int i) -> uint32_t { return sbase + L::OFF_BAR + 8u * (uint32_t)i; };
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::OFF_ABORT);
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + L::OFF_TMEM_PTR);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const Item item = a.items[blockIdx.x / a.heads_per_item];
+    const int h = item.head0 + (int)(blockIdx.x % a.heads_per_item);
+    const int64_t qt = item.q_tile;
+    const int g = h / (a.hq / a.hkv);
+    const Run *rb = a.runs + a.run_off[qt];
+    const Run *re = a.runs + a.run_off[qt + 1];
+    int n = 0;
+    for (const Run *r = rb; r < re; ++r) n += r->kt_end - r->kt_begin;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(bar(L::B_QD), 1);
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(bar(L::B_KV_FULL + i), 1);
+            mbar_init(bar(L::B_KV_EMPTY + i), 1);
+        }
+        mbar_init(bar(L::B_S_FULL), 1);
+        mbar_init(bar(L::B_S_FREE), 256);
+        mbar_init(bar(L::B_DS_READY), 256);
+        mbar_init(bar(L::B_DS_FREE), 1);
+        mbar_init(bar(L::B_DS_FREE + 1), 1);
+        mbar_init(bar(L::B_MMA_DONE), 1);
+        mbar_fence_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 2) {
+        tmem_alloc(smem_u32(tmem_ptr), L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_ptr;
+
+    // k-tile j of this query tile (runs in order)
+    struct Cursor {
+        const Run *r, *end;
+        int32_t kt;
+        __device__ Cursor(const Run *b, const Run *e) : r(b), end(e), kt(b < e ? b->kt_begin : 0) {}
+        __device__ void next() {
+            if (++kt >= r->kt_end) {
+                ++r;
+                if (r < end) kt = r->kt_begin;
+            }
+        }
+    };
+
+    if (warp == 0) {
+        if (lane == 0 && n > 0) {
+            const size_t qtile = ((size_t)h * a.nqt + qt) * (128 * DPAD);
+            mbar_arrive_expect_tx(bar(L::B_QD), 2 * L::TILE);
+            bulk_g2s(sbase + L::OFF_Q, a.qimg16 + qtile, L::TILE, bar(L::B_QD));
+            bulk_g2s(sbase + L::OFF_DO, a.doimg + qtile, L::TILE, bar(L::B_QD));
+            int issued = 0;
+            Cursor cur(rb, re);
+            for (int j = 0; j < n; ++j, cur.next()) {
+                const int s = j % STAGES;
+                if (j >= STAGES &&
+                    !wait_abort(bar(L::B_KV_EMPTY + s), ((j / STAGES) - 1) & 1, a.status, abort_flag, a.timeout_ns))
+                    break;
+                const size_t ktile = ((size_t)g * a.nkt + cur.kt) * (128 * DPAD);
+                mbar_arrive_expect_tx(bar(L::B_KV_FULL + s), 2 * L::TILE);
+                bulk_g2s(sbase + L::OFF_K + s * L::TILE, a.kimg16 + ktile, L::TILE, bar(L::B_KV_FULL + s));
+                bulk_g2s(sbase + L::OFF_V + s * L::TILE, a.vimg + ktile, L::TILE, bar(L::B_KV_FULL + s));
+                ++issued;
+            }
+            // every issued copy must have landed before the CTA may exit
+            for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+                if (!mbar_wait(bar(L::B_KV_FULL + j % STAGES), (j / STAGES) & 1, a.timeout_ns))
+                    atomicOr(a.status, kStatusTimeout);
+            if (!mbar_wait(bar(L::B_QD), 0, a.timeout_ns)) atomicOr(a.status, kStatusTimeout);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0 && n > 0) {
+            const uint64_t dq_k = smem_desc(sbase + L::OFF_Q, 2048, 128);    // Q-hat, K-major A
+            const uint64_t ddo_k = smem_desc(sbase + L::OFF_DO, 2048, 128);  // dO, K-major A
+            const uint64_t dk_k = smem_desc(sbase + L::OFF_K, 2048, 128);    // K-hat, K-major B of S
+            const uint64_t dv_k = smem_desc(sbase + L::OFF_V, 2048, 128);    // V, K-major B of dP
+            const uint64_t dk_mn = smem_desc(sbase + L::OFF_K, 128, 2048);   // K-hat, MN-major B of dQ
+            const uint64_t dds = smem_desc(sbase + L::OFF_DS, 2048, 128);    // dS, K-major A of dQ
+            auto stage_off = [&](int j) -> uint64_t { return (uint64_t)(((j % STAGES) * L::TILE) >> 4); };
+            auto issue_s_dp = [&](int j) {
+                const uint64_t so = stage_off(j);
+#pragma unroll
+                for (int kk = 0; kk < DPAD / 16; ++kk)
+                    mma_f16(tbase + L::COL_S, dq_k + (uint64_t)(kk * 256), dk_k + so + (uint64_t)(kk * 256), IDESC_S,
+                            kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < DPAD / 16; ++kk)
+                    mma_f16(tbase + L::COL_DP, ddo_k + (uint64_t)(kk * 256), dv_k + so + (uint64_t)(kk * 256),
+                            IDESC_DP, kk > 0);
+            };
+            auto issue_dq = [&](int j) {
+                const uint64_t so = stage_off(j), bo = (uint64_t)(((j & 1) * 32768) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16(tbase + L::COL_DQ, dds + bo + (uint64_t)(kk * 256), dk_mn + so + (uint64_t)(kk * 16),
+                            IDESC_DQ, (j > 0 || kk > 0) ? 1u : 0u);
+            };
+            bool ok = wait_abort(bar(L::B_QD), 0, a.status, abort_flag, a.timeout_ns) &&
+                      wait_abort(bar(L::B_KV_FULL), 0, a.status, abort_flag, a.timeout_ns);
+            tc_fence_after();
+            if (ok) {
+                issue_s_dp(0);
+                mma_commit(bar(L::B_S_FULL));
+            }
+            for (int j = 0; j < n && ok; ++j) {
+                if (j + 1 < n) {
+                    ok = wait_abort(bar(L::B_KV_FULL + (j + 1) % STAGES), ((j + 1) / STAGES) & 1, a.status, abort_flag,
+                                    a.timeout_ns) &&
+                         wait_abort(bar(L::B_S_FREE), j & 1, a.status, abort_flag, a.timeout_ns);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_s_dp(j + 1);
+                    mma_commit(bar(L::B_S_FULL));
+                }
+                ok = wait_abort(bar(L::B_DS_READY), j & 1, a.status, abort_flag, a.timeout_ns);
+                if (!ok) break;
+                tc_fence_after();
+                issue_dq(j);
+                mma_commit(bar(L::B_DS_FREE + (j & 1)));
+                mma_commit(bar(L::B_KV_EMPTY + j % STAGES));
+            }
+            mma_commit(bar(L::B_MMA_DONE));
+            if (!mbar_wait(bar(L::B_MMA_DONE), 0, a.timeout_ns)) {
+                atomicOr(a.status, kStatusTimeout);
+                *abort_flag = 1;
+            }
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        const int half = (warp - 4) / 4;  // key columns [64 half, 64 half + 64)
+        const int quarter = warp % 4;
+        const int row = quarter * 32 + lane;
+        const int c0 = 64 * half;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const size_t vec = ((size_t)h * a.nqt + qt) * 128 + row;
+        const float nlse = a.lse2[vec], ndsum = a.dsum[vec];  // -LSE2 (+ log2 sc) and -Dsum of this row
+        uint4 *dsb0 = reinterpret_cast<uint4 *>(smem + L::OFF_DS);
+        bool ok = true;
+        Cursor cur(rb, re);
+        for (int j = 0; j < n; ++j, cur.next()) {
+            ok = warp_wait_abort(bar(L::B_S_FULL), j & 1, a.status, abort_flag, a.timeout_ns);
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sv[64], pv[64];
+            tmem_ld32(tbase + lane_off + L::COL_S + c0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+            tmem_ld32(tbase + lane_off + L::COL_S + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+            tmem_ld32(tbase + lane_off + L::COL_DP + c0, *reinterpret_cast<uint32_t(*)[32]>(&pv[0]));
+            tmem_ld32(tbase + lane_off + L::COL_DP + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pv[32]));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(bar(L::B_S_FREE));
+            const int b = j & 1;
+            if (j > 1) {  // dS buffer b was last read by the dQ MMAs of tile j - 2
+                ok = warp_wait_abort(bar(L::B_DS_FREE + b), ((j >> 1) - 1) & 1, a.status, abort_flag, a.timeout_ns);
+                if (!ok) break;
+            }
+            uint32_t mw0 = 0xffffffffu, mw1 = 0xffffffffu;
+            if (cur.r->mask_idx >= 0) {
+                const uint32_t *mk = a.masks + ((size_t)cur.r->mask_idx * 128 + row) * 4;
+                mw0 = mk[c0 / 32];
+                mw1 = mk[c0 / 32 + 1];
+            }
+            uint4 *dsb = dsb0 + b * 2048;
+            const float2 nl = make_float2(nlse, nlse), nd = make_float2(ndsum, ndsum);
+#pragma unroll
+            for (int k8 = 0; k8 < 8; ++k8) {  // 8 keys per 16-byte chunk
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c = 8 * k8 + 2 * e;
+                    const float2 x = __fadd2_rn(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), nl);
+                    float2 p = make_float2(ex2(x.x), ex2(x.y));
+                    const uint32_t mw = c < 32 ? mw0 : mw1;
+                    if (!((mw >> (c % 32)) & 1u)) p.x = 0.f;
+                    if (!((mw >> ((c + 1) % 32)) & 1u)) p.y = 0.f;
+                    const float2 t = __fadd2_rn(make_float2(__uint_as_float(pv[c]), __uint_as_float(pv[c + 1])), nd);
+                    const float2 ds = __fmul2_rn(p, t);
+                    w[e] = pack_f16x2(ds.x, ds.y);
+                }
+                dsb[img_chunk(c0 / 8 + k8, row)] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(L::B_DS_READY));
+        }
+        // dQ-hat sc of this row and column half: every element is written (zeros when the
+        // query tile sees no key), so the accumulator needs no clearing
+        float acc[HALF];
+#pragma unroll
+        for (int c = 0; c < HALF; ++c) acc[c] = 0.f;
+        if (n > 0 && ok) ok = warp_wait_abort(bar(L::B_MMA_DONE), 0, a.status, abort_flag, a.timeout_ns);
+        tc_fence_after();
+        if (n > 0 && ok) {
+#pragma unroll
+            for (int c = 0; c < HALF / 8; ++c) {
+                uint32_t r8[8];
+                tmem_ld8(tbase + lane_off + L::COL_DQ + half * HALF + 8 * c, r8);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[8 * c + e] = __uint_as_float(r8[e]);
+            }
+        }
+        float4 *dst = reinterpret_cast<float4 *>(a.dqacc + ((((size_t)h * a.nqt + qt) * 2 + half) * 128 + row) * HALF);
+#pragma unroll
+        for (int c = 0; c < HALF / 4; ++c)
+            dst[c] = make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
     }
 
     tc_fence_before();
@@ -821,7 +1120,8 @@ __global__ void __launch_bounds__(128) bwd_dq_kernel(DqArgs a) {
         if (want_pg)
             qk_param_grads<D>(x, g, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps, a.coef,
                               __ldg(a.tbase), pg, pb);
-        qk_prologue_bwd<D>(x, g, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps);
+        qk_prologue_bwd<D>(x, g, __ldg(a.pos + q), a.q_gain, a.rope, a.off0, a.off1, a.off2, a.eps,
+                           a.prologue != 0);
         float *dst = a.dq + row * D;
 #pragma unroll
         for (int c = 0; c < D / 4; ++c)
@@ -875,7 +1175,9 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     auto *bounds = reinterpret_cast<float *>(ws + 2 * kvb + 2 * qb + 2 * vb);
     auto *dqacc = reinterpret_cast<float *>(ws + 2 * kvb + 2 * qb + 2 * vb + 256);
     if (cudaMemsetAsync(bounds, 0, 2 * sizeof(float), stream) != cudaSuccess) return BCA_ERR_CUDA;
-    if (cudaMemsetAsync(dqacc, 0, dq_acc_bytes(P), stream) != cudaSuccess) return BCA_ERR_CUDA;
+    const bool dq_pass = (P.flags & BCA_DQ_DETERMINISTIC) != 0;
+    // the reduce-adds need a zeroed accumulator; the deterministic pass writes every element
+    if (!dq_pass && cudaMemsetAsync(dqacc, 0, dq_acc_bytes(P), stream) != cudaSuccess) return BCA_ERR_CUDA;
     // parameter gradients are sums over rows: start them at zero
     if (io.dq_gain && cudaMemsetAsync(io.dq_gain, 0, D * sizeof(float), stream) != cudaSuccess) return BCA_ERR_CUDA;
     if (io.dk_gain && cudaMemsetAsync(io.dk_gain, 0, D * sizeof(float), stream) != cudaSuccess) return BCA_ERR_CUDA;
@@ -899,6 +1201,7 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     pa.hq = P.hq;
     pa.eps = P.eps;
     pa.qscale = kLog2e / sqrtf((float)D);
+    pa.prologue = (P.flags & BCA_NO_PROLOGUE) ? 0 : 1;
     pa.qimg16 = qimg16;
     pa.doimg = doimg;
     pa.bounds = bounds;
@@ -926,6 +1229,8 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     ka.nkt = P.nkt;
     ka.hkv = P.hkv;
     ka.eps = P.eps;
+    ka.prologue = (P.flags & BCA_NO_PROLOGUE) ? 0 : 1;
+    ka.kc_f16 = (P.flags & BCA_CACHE_K_FP16) ? 1 : 0;
     ka.kimg16 = kimg16;
     ka.vimg = vimg;
     ka.bounds = bounds;
@@ -971,6 +1276,7 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     ba.hq = P.hq;
     ba.hkv = P.hkv;
     ba.eps = P.eps;
+    ba.prologue = (P.flags & BCA_NO_PROLOGUE) ? 0 : 1;
     ba.dqacc = dqacc;
     ba.dk = io.dk;
     ba.dv = io.dv;
@@ -982,11 +1288,39 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     ba.tbase = P.d_tbase;
     ba.accumulate = io.accumulate;
     ba.status = P.d_status;
+    ba.timeout_ns = (P.flags & BCA_TEST_FORCE_TIMEOUT) ? 1000000ull : kWaitTimeoutNs;
+    ba.skip_loads = (P.flags & BCA_TEST_FORCE_TIMEOUT) ? 1 : 0;
+    ba.dq_pass = dq_pass ? 1 : 0;
     {
         ProfScope ps(P, BCA_KERNEL_BWD, stream);
         bwd_kernel<D><<<(unsigned)P.bwd_items.size(), 384, L::BYTES, stream>>>(ba);
     }
     if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
+
+    if (dq_pass) {
+        DqPassArgs qa;
+        qa.kimg16 = kimg16;
+        qa.qimg16 = qimg16;
+        qa.vimg = vimg;
+        qa.doimg = doimg;
+        qa.lse2 = lse2;
+        qa.dsum = dsum;
+        qa.items = P.d_items;
+        qa.run_off = P.d_run_off;
+        qa.runs = P.d_runs;
+        qa.masks = P.d_masks;
+        qa.nqt = P.nqt;
+        qa.nkt = P.nkt;
+        qa.hq = P.hq;
+        qa.hkv = P.hkv;
+        qa.heads_per_item = P.heads_per_item;
+        qa.dqacc = dqacc;
+        qa.status = P.d_status;
+        qa.timeout_ns = ba.timeout_ns;
+        ProfScope ps(P, BCA_KERNEL_BWD_DQ_PASS, stream);
+        bwd_dq_pass_kernel<D><<<(unsigned)(P.items.size() * P.heads_per_item), 384, DqSmem<D>::BYTES, stream>>>(qa);
+        if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
+    }
 
     DqArgs da;
     da.q = static_cast<const __nv_bfloat16 *>(io.q);
@@ -1001,6 +1335,7 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
     da.hq = P.hq;
     da.eps = P.eps;
     da.scale = 1.0f / sqrtf((float)D);
+    da.prologue = (P.flags & BCA_NO_PROLOGUE) ? 0 : 1;
     da.dq = io.dq;
     da.dqacc = dqacc;
     da.bounds = bounds;
@@ -1043,9 +1378,18 @@ int prepare_bwd(const Plan &P) {
     };
     bool ok = true;
     switch (P.d) {
-        case 24: ok = set((const void *)bwd_kernel<24>, BwdSmem<24>::BYTES); break;
-        case 32: ok = set((const void *)bwd_kernel<32>, BwdSmem<32>::BYTES); break;
-        case 48: ok = set((const void *)bwd_kernel<48>, BwdSmem<48>::BYTES); break;
+        case 24:
+            ok = set((const void *)bwd_kernel<24>, BwdSmem<24>::BYTES) &&
+                 set((const void *)bwd_dq_pass_kernel<24>, DqSmem<24>::BYTES);
+            break;
+        case 32:
+            ok = set((const void *)bwd_kernel<32>, BwdSmem<32>::BYTES) &&
+                 set((const void *)bwd_dq_pass_kernel<32>, DqSmem<32>::BYTES);
+            break;
+        case 48:
+            ok = set((const void *)bwd_kernel<48>, BwdSmem<48>::BYTES) &&
+                 set((const void *)bwd_dq_pass_kernel<48>, DqSmem<48>::BYTES);
+            break;
         default: return BCA_ERR_UNSUPPORTED;
     }
     return ok ? BCA_OK : BCA_ERR_CUDA;

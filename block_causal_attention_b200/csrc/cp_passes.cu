@@ -29,6 +29,8 @@ struct RowArgs {
     int64_t rows;  // tokens * heads
     int heads;
     float eps;
+    int prologue;            // 0: keys given post-prologue (BCA_NO_PROLOGUE): both passes copy
+    int khat_f16;            // write K-hat as fp16 (BCA_CACHE_K_FP16), else bf16
     __nv_bfloat16 *k_hat;    // forward output
     const float *dk_hat;     // backward input
     float *dk;               // backward output
@@ -42,10 +44,10 @@ __global__ void __launch_bounds__(128) k_prologue_kernel(RowArgs a) {
     const int64_t t = row / a.heads;
     float x[D];
     load_row_bf16<D>(a.k + (size_t)row * D, x);
-    qk_prologue<D>(x, __ldg(a.pos + t), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps, 1.0f);
+    qk_prologue<D>(x, __ldg(a.pos + t), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps, 1.0f, a.prologue != 0);
     uint4 *dst = reinterpret_cast<uint4 *>(a.k_hat + (size_t)row * D);
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) dst[c] = pack_chunk_bf16<D>(x, c);
+    for (int c = 0; c < D / 8; ++c) dst[c] = a.khat_f16 ? pack_chunk_f16<D>(x, c) : pack_chunk_bf16<D>(x, c);
 }
 
 template <int D>
@@ -64,7 +66,7 @@ __global__ void __launch_bounds__(128) k_prologue_bwd_kernel(RowArgs a) {
         g[4 * c + 2] = f.z;
         g[4 * c + 3] = f.w;
     }
-    qk_prologue_bwd<D>(x, g, __ldg(a.pos + t), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps);
+    qk_prologue_bwd<D>(x, g, __ldg(a.pos + t), a.k_gain, a.rope, a.off0, a.off1, a.off2, a.eps, a.prologue != 0);
     float4 *dst = reinterpret_cast<float4 *>(a.dk + (size_t)row * D);
 #pragma unroll
     for (int c = 0; c < D / 4; ++c) {
@@ -92,6 +94,8 @@ RowArgs row_args(const Plan &P, const void *k, const float *k_gain) {
     a.rows = P.nq * P.hkv;
     a.heads = P.hkv;
     a.eps = P.eps;
+    a.prologue = (P.flags & BCA_NO_PROLOGUE) ? 0 : 1;
+    a.khat_f16 = (P.flags & BCA_CACHE_K_FP16) ? 1 : 0;
     return a;
 }
 

@@ -52,6 +52,7 @@ extern "C" int bca_fwd_static_workspace(bca_plan_t plan, const void *q, const vo
     if (bca::fwd_workspace_bytes(P) > (size_t)BCA_STATIC_WORKSPACE_BYTES) return BCA_ERR_TOO_LARGE;
     if (!q || !k || !v || !o || !lse) return BCA_ERR_INVALID_ARGUMENT;
     if (P.nc > 0 && (!k_cache || !v_cache)) return BCA_ERR_INVALID_ARGUMENT;
+    if ((P.flags & BCA_NO_PROLOGUE) && (q_gain || k_gain)) return BCA_ERR_INVALID_ARGUMENT;
     const void *ptrs[] = {q, k, v, k_cache, v_cache, q_gain, k_gain, o, lse};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return BCA_ERR_MISALIGNED;

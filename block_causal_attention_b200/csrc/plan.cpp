@@ -121,11 +121,12 @@ void compile_q_tile(const Plan &P, int64_t qt, TileOut &out) {
 
 int validate_problem(const bca_problem *p, Plan &P) {
     if (!p) return BCA_ERR_INVALID_ARGUMENT;
-    if (p->flags & ~(BCA_O_FP32 | BCA_PLAN_HOST_ONLY | BCA_TEST_FORCE_TIMEOUT | BCA_FWD_FP8_E4M3))
+    if (p->flags & ~(BCA_O_FP32 | BCA_PLAN_HOST_ONLY | BCA_TEST_FORCE_TIMEOUT | BCA_FWD_FP8_E4M3 | BCA_NO_PROLOGUE |
+                     BCA_DQ_DETERMINISTIC | BCA_CACHE_K_FP16))
         return BCA_ERR_INVALID_ARGUMENT;
+    if ((p->flags & BCA_FWD_FP8_E4M3) && (p->flags & (BCA_NO_PROLOGUE | BCA_CACHE_K_FP16))) return BCA_ERR_UNSUPPORTED;
     if (p->num_q_heads <= 0 || p->num_kv_heads <= 0) return BCA_ERR_INVALID_ARGUMENT;
     if (p->num_q_heads % p->num_kv_heads != 0) return BCA_ERR_UNSUPPORTED;
-    if ((p->num_q_heads / p->num_kv_heads) % 2 != 0) return BCA_ERR_UNSUPPORTED;
     if (p->head_dim != 24 && p->head_dim != 32 && p->head_dim != 48) return BCA_ERR_UNSUPPORTED;
     if (p->num_videos < 0 || (p->num_videos > 0 && !p->videos)) return BCA_ERR_INVALID_ARGUMENT;
     if (p->num_cache_keys < 0) return BCA_ERR_INVALID_ARGUMENT;
@@ -275,7 +276,9 @@ int compile_plan(Plan &P) {
     // ---- items, longest first; ties grouped by KV group then q-tile so that CTAs
     //      running together stream the same K/V tiles ----
     const int G = P.hq / P.hkv;
-    P.heads_per_item = 2;
+    // two query heads of one KV group per forward CTA share each K/V tile; an odd group
+    // size (MHA included) runs one head per CTA
+    P.heads_per_item = (G % 2 == 0) ? 2 : 1;
     const int nsets = P.hq / P.heads_per_item;
     P.items.clear();
     P.items.reserve((size_t)P.nqt * nsets);

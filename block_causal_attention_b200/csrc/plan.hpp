@@ -28,7 +28,7 @@ struct Item {
 struct Plan {
     // problem
     int hq = 0, hkv = 0, d = 0, dpad = 0;
-    int heads_per_item = 2;  // query heads per forward CTA: 4 when the group size allows
+    int heads_per_item = 2;  // query heads per forward CTA: 2, or 1 for an odd group size
     int64_t nq = 0, nk = 0, nc = 0;
     uint32_t flags = 0;
     float base[3] = {1e4f, 1e4f, 1e4f};

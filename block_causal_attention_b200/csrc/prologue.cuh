@@ -29,11 +29,19 @@ struct Geo {
 
 // ------------------------------------------------------------------ prologue math
 
-// RMS QK-Norm with gain, 3D RoPE at the packed position, then a scale; in place.
+// RMS QK-Norm with gain, 3D RoPE at the packed position, then a scale; in place.  With
+// apply = false (plans created with BCA_NO_PROLOGUE: the rows are given post-prologue)
+// only the scale is applied.
 template <int D>
 __device__ __forceinline__ void qk_prologue(float (&x)[D], uint32_t pos, const float *gain, const float *rope,
-                                            int32_t off0, int32_t off1, int32_t off2, float eps, float scale) {
+                                            int32_t off0, int32_t off1, int32_t off2, float eps, float scale,
+                                            bool apply = true) {
     constexpr int P = Geo<D>::PAIRS;
+    if (!apply) {
+#pragma unroll
+        for (int d = 0; d < D; ++d) x[d] *= scale;
+        return;
+    }
     float ss = 0.f;
 #pragma unroll
     for (int d = 0; d < D; ++d) ss = fmaf(x[d], x[d], ss);
@@ -68,6 +76,28 @@ __device__ __forceinline__ void load_row_bf16(const __nv_bfloat16 *src, float (&
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             float2 f = __bfloat1622float2(b[e]);
+            x[c * 8 + 2 * e] = f.x;
+            x[c * 8 + 2 * e + 1] = f.y;
+        }
+    }
+}
+
+// A row of 16-bit values: bf16, or fp16 when f16 (cache keys of plans created with
+// BCA_CACHE_K_FP16).
+template <int D>
+__device__ __forceinline__ void load_row_16(const void *src, bool f16, float (&x)[D]) {
+    if (!f16) {
+        load_row_bf16<D>(static_cast<const __nv_bfloat16 *>(src), x);
+        return;
+    }
+    const uint4 *s = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+        uint4 u = __ldg(s + c);
+        const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float2 f = __half22float2(h[e]);
             x[c * 8 + 2 * e] = f.x;
             x[c * 8 + 2 * e + 1] = f.y;
         }
@@ -110,11 +140,13 @@ __device__ __forceinline__ uint4 pack_chunk_e4m3(const float (&x)[D], int c, flo
 // Backward of qk_prologue (with scale 1) for one row: g holds dL/d(output) on entry
 // and dL/dx on exit; x is the raw input row.  RoPE^T rotates by -angle; the
 // RMS-norm backward is dx = gain*dz*r - x * sum(gain*dz*x) * r^3 / D, r = 1/rms.
+// With apply = false (no prologue) the gradient passes through unchanged.
 template <int D>
 __device__ __forceinline__ void qk_prologue_bwd(const float (&x)[D], float (&g)[D], uint32_t pos, const float *gain,
                                                 const float *rope, int32_t off0, int32_t off1, int32_t off2,
-                                                float eps) {
+                                                float eps, bool apply = true) {
     constexpr int P = Geo<D>::PAIRS;
+    if (!apply) return;
     const int32_t p[3] = {(int32_t)(pos >> 16), (int32_t)((pos >> 8) & 255u), (int32_t)(pos & 255u)};
     const int32_t off[3] = {off0, off1, off2};
 #pragma unroll

@@ -72,9 +72,11 @@ extern "C" {
 /* bca_problem.flags */
 #define BCA_O_FP32 0x1u          /* write O as fp32 instead of bf16 */
 #define BCA_PLAN_HOST_ONLY 0x2u  /* compile the mask on the host only (no CUDA calls) */
-#define BCA_TEST_FORCE_TIMEOUT 0x4u /* failure-detection test: bca_fwd's K/V loads are not
-                                       issued and its waits give up after 1 ms, so every
-                                       CTA records BCA_ERR_DEVICE_TIMEOUT and exits cleanly */
+#define BCA_TEST_FORCE_TIMEOUT 0x4u /* failure-detection test: the attention kernels of bca_fwd
+                                       and bca_bwd issue none of their tile loads and their
+                                       waits give up after 1 ms, so every CTA records
+                                       BCA_ERR_DEVICE_TIMEOUT and exits cleanly (outputs are
+                                       then meaningless) */
 #define BCA_FWD_FP8_E4M3 0x8u /* forward with e4m3 tensor-core operands (the 8-bit float
                                  MMAs of sm_100a): Q-hat and K-hat rounded to e4m3, V to
                                  e4m3 after division by a power of two per KV head (from
@@ -89,6 +91,31 @@ extern "C" {
                                  number of keys), not to bf16 precision.  Forward only:
                                  bca_bwd / bca_bwd_ex on such a plan return
                                  BCA_ERR_UNSUPPORTED (train with bf16 plans). */
+#define BCA_NO_PROLOGUE 0x10u /* q and k are given post-prologue: no QK-Norm and no RoPE
+                                 is applied (the attention alone, s = q.k / sqrt(D)), and
+                                 the gradients are w.r.t. the given q and k.  The kernels
+                                 stage q and k as fp16 (11-bit significand), so every
+                                 element must satisfy |x| < 60000 (else it rounds to
+                                 infinity).  q_gain, k_gain and the parameter gradients of
+                                 bca_bwd_ex do not exist then: passing any of them returns
+                                 BCA_ERR_INVALID_ARGUMENT.  bca_k_prologue copies k (bf16)
+                                 and bca_k_prologue_bwd passes dk_hat through.  Not
+                                 combinable with BCA_FWD_FP8_E4M3 (BCA_ERR_UNSUPPORTED). */
+#define BCA_DQ_DETERMINISTIC 0x20u /* bca_bwd / bca_bwd_ex form dQ by a separate pass, one CTA
+                                      per (query tile, query head) walking its key tiles in a
+                                      fixed order (S and dP are recomputed there), instead of
+                                      summing the key-tile CTAs' shares with reduce-adds whose
+                                      order varies: dQ is then bit-identical from run to run,
+                                      like dK and dV.  Costs two more matrix products per
+                                      visible tile.  (The parameter gradients of bca_bwd_ex
+                                      still use atomic adds.) */
+#define BCA_CACHE_K_FP16 0x40u /* k_cache is IEEE fp16 instead of bf16, and bca_k_prologue
+                                  writes fp16 K-hat.  The kernels stage K-hat as fp16
+                                  anyway, so a cache key given in fp16 enters the scores
+                                  with the same rounding as a new key of the plan; context
+                                  parallelism uses this for keys borrowed from other ranks.
+                                  Cache keys must then stay below 65,504 in magnitude.
+                                  Not combinable with BCA_FWD_FP8_E4M3. */
 
 /* bca_workspace_bytes(pass) */
 #define BCA_PASS_FWD 0
@@ -109,7 +136,9 @@ typedef struct {
 
 typedef struct {
     int32_t num_q_heads;        /* Hq */
-    int32_t num_kv_heads;       /* Hkv; Hq % Hkv == 0 and (Hq / Hkv) even */
+    int32_t num_kv_heads;       /* Hkv; Hq % Hkv == 0.  An even group size Hq / Hkv runs two
+                                   query heads per forward work item (each K/V tile loaded
+                                   once for both), an odd one (MHA, Hkv = Hq, included) one */
     int32_t head_dim;           /* D in {24, 32, 48} */
     int32_t num_videos;
     const bca_video *videos;    /* Nq = sum of chunks*frames*height*width */
@@ -120,7 +149,8 @@ typedef struct {
     float rope_base[3];         /* RoPE base per axis (t, h, w) */
     float norm_eps;             /* QK-Norm epsilon */
     uint32_t flags;             /* BCA_O_FP32 | BCA_PLAN_HOST_ONLY | BCA_TEST_FORCE_TIMEOUT |
-                                   BCA_FWD_FP8_E4M3 */
+                                   BCA_FWD_FP8_E4M3 | BCA_NO_PROLOGUE | BCA_DQ_DETERMINISTIC |
+                                   BCA_CACHE_K_FP16 */
 } bca_problem;
 
 typedef struct bca_plan_s *bca_plan_t;
@@ -131,7 +161,8 @@ typedef struct {
     int64_t num_q_tiles, num_k_tiles;
     int64_t num_runs;            /* runs of consecutive k-tiles over all q-tiles */
     int64_t num_full_tiles, num_partial_tiles;
-    int64_t num_items;           /* forward work items (q-tile x 2 or 4 heads of a group) */
+    int64_t num_items;           /* forward work items (q-tile x 2 query heads of one KV
+                                    group, or x 1 head for an odd group size) */
     int64_t visible_pairs;       /* visible (query, key) pairs per head */
     int32_t head_dim_padded;     /* D rounded up to the MMA k-granule (16) */
     int32_t tile_q, tile_k;
@@ -177,7 +208,8 @@ int bca_plan_update_positions(bca_plan_t plan, const bca_video *videos, int num_
  * BCA_FWD_FP8_E4M3 plans the smaller e4m3 images plus one float of max|V| per KV head. */
 size_t bca_workspace_bytes(bca_plan_t plan, int pass);
 
-/* Forward.  q, k, v, k_cache, v_cache: bf16 (k_cache/v_cache NULL iff Nc == 0);
+/* Forward.  q, k, v, k_cache, v_cache: bf16 (k_cache fp16 for BCA_CACHE_K_FP16 plans;
+ * k_cache/v_cache NULL iff Nc == 0);
  * q_gain, k_gain: fp32 [D] QK-Norm gains or NULL (= ones); o: bf16 or fp32
  * (BCA_O_FP32) [Nq][Hq][D]; lse: fp32 [Hq][Nq]; workspace: bca_workspace_bytes(FWD)
  * bytes; stream: a cudaStream_t (NULL = legacy default stream). */
@@ -224,7 +256,8 @@ int bca_fwd_static_workspace(bca_plan_t plan, const void *q, const void *k, cons
  * [Nc][Hkv][D] (cache keys are used as given, so their gradient is taken at the
  * rotated keys; NULL = not wanted).  workspace: bca_workspace_bytes(BWD) bytes.
  * dk, dv, dk_cache and dv_cache are reduced in a fixed order (bit-reproducible run to
- * run); dq is accumulated with atomics, so its last bits may vary between runs. */
+ * run); dq is accumulated with atomics, so its last bits may vary between runs, unless
+ * the plan was created with BCA_DQ_DETERMINISTIC. */
 int bca_bwd(bca_plan_t plan, const void *q, const void *k, const void *v,
             const void *k_cache, const void *v_cache, const float *q_gain,
             const float *k_gain, const void *o, const float *lse, const void *dout,
@@ -269,7 +302,7 @@ int bca_attn_merge(bca_plan_t plan, const float *o_a, const float *lse_a, const 
  * key are mapped back through the prologue by the owner (MAGI-1 research notes,
  * "Infra > MagiAttention": group-cast and group-reduce).
  *   k      : bf16 [Nq][Hkv][D], the plan's new tokens' raw keys; k_gain: fp32 [D] or NULL;
- *   k_hat  : bf16 [Nq][Hkv][D] out (RNE of the fp32 result);
+ *   k_hat  : bf16 [Nq][Hkv][D] out (RNE of the fp32 result; fp16 for BCA_CACHE_K_FP16 plans);
  *   dk_hat : fp32 [Nq][Hkv][D], dL/dk_hat;  dk: fp32 [Nq][Hkv][D] out, overwritten, or
  *            added to when accumulate != 0.
  * 16-byte aligned pointers; asynchronous on `stream`. */
@@ -284,7 +317,8 @@ int bca_k_prologue_bwd(bca_plan_t plan, const void *k, const float *k_gain, cons
 #define BCA_KERNEL_BWD_KV_IMAGE 3  /* K-hat / V images for the backward */
 #define BCA_KERNEL_BWD 4           /* attention backward */
 #define BCA_KERNEL_BWD_DQ 5        /* dQ prologue backward */
-#define BCA_KERNEL_COUNT 6
+#define BCA_KERNEL_BWD_DQ_PASS 6   /* deterministic dQ pass (BCA_DQ_DETERMINISTIC) */
+#define BCA_KERNEL_COUNT 7
 
 /* Per-kernel device timing, a tracing aid.  While enabled (enable != 0), every
  * kernel that bca_fwd or bca_bwd launches for this plan is bracketed by two CUDA events

@@ -146,13 +146,30 @@ def test_bwd_large_upstream_gradient(name):
 
 
 @pytest.mark.parametrize("name,nrows", [("p720_pipelined", 24), ("packed_varlen", 24), ("long_kvrange", 12)])
-def test_bwd_full_size_sampled_dq_and_dv_sums(name, nrows):
-    """Full-size workloads in the benchmark's launch configuration: dq on a seeded row
-    sample computed exactly by the oracle; and, per KV group, sum_j dV_j equals the sum
-    of dO over the group's heads (rows of P sum to one)."""
+def test_bwd_full_size_sampled_rows_and_key_rows(name, nrows):
+    """Full-size workloads in the benchmark's launch configuration:
+    * dK and dV (and dK_cache, dV_cache) of seeded key rows of one KV group, element by
+      element, against the fp64 oracle's values stored in tests/golden/key_grads_<name>.npz
+      (written by tests/golden/make_key_grads.py from the oracle alone; the keys include
+      chunk edges, cache keys and keys that transition chunks see);
+    * dq on a seeded row sample computed exactly by the oracle;
+    * per KV group, sum_j dV_j equals the sum of dO over the group's heads (rows of P sum
+      to one), an extra whole-tensor check."""
+    import os
     w = W.WORKLOADS[name]
     x = W.make_inputs(w, "cuda", with_grad=True)
     dq, dk, dv, dkc, dvc = _gpu_fwd_bwd(w, x)
+    gold = np.load(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", f"key_grads_{name}.npz"))
+    keys, g, nc = gold["keys"], int(gold["group"]), w.num_cache_keys
+    new, old = keys >= nc, keys < nc
+    assert new.any()
+    kn = torch.as_tensor(keys[new] - nc, device="cuda")
+    print(name, _err("dk key rows", dk[kn, g], gold["dk"][new].astype(np.float64)),
+          _err("dv key rows", dv[kn, g], gold["dv"][new].astype(np.float64)))
+    if old.any():
+        ko = torch.as_tensor(keys[old], device="cuda")
+        print(name, _err("dk_cache key rows", dkc[ko, g], gold["dk"][old].astype(np.float64)),
+              _err("dv_cache key rows", dvc[ko, g], gold["dv"][old].astype(np.float64)))
     rows = W.sample_rows(w, nrows)
     xc = {k: (None if t is None else t.cpu()) for k, t in x.items() if k in ("k", "v", "k_cache", "v_cache")}
     rq = oracle.backward_rows(W.make_input_rows(w, W.T_Q, rows), rows, xc["k"], xc["v"], xc["k_cache"],
@@ -186,3 +203,29 @@ def test_bwd_full_size_sampled_key_rows(name, groups):
     for g in groups:
         rk, rv = video_key_grads(w, 0, g, keys)
         print(name, g, _err("dk rows", dk[kr, g], rk), _err("dv rows", dv[kr, g], rv))
+
+
+@pytest.mark.parametrize("name", ["tiny", "p720_replica", "kvrange_replica", "b45_replica"])
+def test_bwd_deterministic_dq_pass(name):
+    """BCA_DQ_DETERMINISTIC: dQ from the separate fixed-order pass is bit-identical over
+    two runs, matches the oracle, and agrees with the reduce-add path to fp32 rounding;
+    dK and dV are the same as without the flag, bit for bit."""
+    w = W.WORKLOADS[name]
+    x = W.make_inputs(w, "cuda", with_grad=True)
+    pd = Plan(w.hq, w.hkv, w.d, w.videos_array(), w.num_cache_keys, w.slices_array(), w.rope_base, w.eps, w.o_fp32,
+              dq_deterministic=True)
+    a = _gpu_fwd_bwd(w, x, pd)
+    b = _gpu_fwd_bwd(w, x, pd)
+    for i in range(5):
+        if a[i] is not None:
+            assert torch.equal(a[i], b[i]), i
+    ref = _gpu_fwd_bwd(w, x, Plan.from_workload(w))
+    for i in (1, 2, 3, 4):
+        if a[i] is not None:
+            assert torch.equal(a[i], ref[i]), i
+    assert (a[0] - ref[0]).abs().max().item() <= 1e-5
+    c = {k: (None if t is None else t.cpu()) for k, t in x.items()}
+    rq, _, _, _, _, _, _ = oracle.backward(c["q"], c["k"], c["v"], c["k_cache"], c["v_cache"], c["do"],
+                                           w.videos_array(), w.slices_array(), w.hq, w.hkv, base=w.rope_base,
+                                           eps=w.eps)
+    print(name, _err("dq (deterministic pass)", a[0], rq))

@@ -144,7 +144,14 @@ def test_argument_checks_return_codes():
     E = _abi
     assert _create() == E.BCA_OK
     assert _create(hq=6, hkv=4) == E.BCA_ERR_UNSUPPORTED           # Hq % Hkv != 0
-    assert _create(hq=6, hkv=2) == E.BCA_ERR_UNSUPPORTED           # odd group size
+    assert _create(hq=6, hkv=2) == E.BCA_OK                        # odd group size: one head per item
+    assert _create(hq=4, hkv=4) == E.BCA_OK                        # MHA
+    H = E.BCA_PLAN_HOST_ONLY
+    assert _create(flags=H | E.BCA_NO_PROLOGUE) == E.BCA_OK
+    assert _create(flags=H | E.BCA_NO_PROLOGUE | E.BCA_FWD_FP8_E4M3) == E.BCA_ERR_UNSUPPORTED
+    assert _create(flags=H | E.BCA_DQ_DETERMINISTIC) == E.BCA_OK
+    assert _create(flags=H | E.BCA_CACHE_K_FP16) == E.BCA_OK
+    assert _create(flags=H | E.BCA_CACHE_K_FP16 | E.BCA_FWD_FP8_E4M3) == E.BCA_ERR_UNSUPPORTED
     assert _create(d=64) == E.BCA_ERR_UNSUPPORTED
     assert _create(d=40) == E.BCA_ERR_UNSUPPORTED
     assert _create(hq=0) == E.BCA_ERR_INVALID_ARGUMENT
