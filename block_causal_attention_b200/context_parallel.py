@@ -291,15 +291,20 @@ class ContextParallelPlan:
 # ----------------------------------------------------------------------------- runtime
 
 def _default_engine(hq, hkv, d, videos, num_cache_keys, slices, rope_base, eps, o_fp32):
+    """CUDA plans whose cache keys (the global cache's and the borrowed ones) are fp16:
+    the owner's K-hat reaches the kernels with the same fp16 rounding as a key of the
+    plan's own tokens, instead of passing through bf16 on the way."""
     from . import Plan
-    return Plan(hq, hkv, d, videos, num_cache_keys, slices, rope_base, eps, o_fp32)
+    return Plan(hq, hkv, d, videos, num_cache_keys, slices, rope_base, eps, o_fp32, cache_k_fp16=True)
 
 
 def _host_staged(group, t) -> bool:
-    """True when the collectives of `group` cannot take `t` where it lives: device tensors
-    on a gloo group (gloo moves host memory), which are then exchanged through host copies."""
+    """True when the collectives of `group` cannot take `t` as it is: device tensors on a
+    gloo group (gloo moves host memory) go through host copies, and 16-bit words (which
+    gloo has no type for) travel in pairs as 32-bit words."""
+    import torch
     import torch.distributed as dist
-    return t.is_cuda and dist.get_backend(group) == "gloo"
+    return dist.get_backend(group) == "gloo" and (t.is_cuda or t.dtype == torch.int16)
 
 
 def _all_to_all_rows(group, send: List, recv_counts: List[int], row_shape, like, async_op: bool = False):
@@ -320,10 +325,15 @@ def _all_to_all_rows(group, send: List, recv_counts: List[int], row_shape, like,
     if world == 1:
         rview.copy_(sview)
     elif _host_staged(group, sview):
-        rhost = torch.empty(rview.shape, dtype=rview.dtype)
-        dist.all_to_all_single(rhost, sview.cpu(), output_split_sizes=list(recv_counts),
+        # gloo has no 16-bit integer type: 16-bit rows (an even count per row) travel as
+        # pairs packed into 32-bit words, still bit-exact
+        pack = sview.dtype == torch.int16
+        shost = sview.cpu()
+        shost = shost.view(torch.int32) if pack else shost
+        rhost = torch.empty((rview.shape[0], shost.shape[1]), dtype=shost.dtype)
+        dist.all_to_all_single(rhost, shost, output_split_sizes=list(recv_counts),
                                input_split_sizes=[int(f.shape[0]) for f in flat], group=group)
-        rview.copy_(rhost)
+        rview.copy_(rhost.view(torch.int16) if pack else rhost)
     else:
         work = dist.all_to_all_single(rview, sview, output_split_sizes=list(recv_counts),
                                       input_split_sizes=[int(f.shape[0]) for f in flat], group=group,
@@ -400,8 +410,12 @@ class ContextParallelAttention:
 
     def _gather_keys_start(self, khat_local, v_local):
         """Send the rows of [K-hat | V] of this rank's tokens that the other ranks need;
-        returns a handle for _gather_keys_finish (the receive may still be in flight)."""
+        returns a handle for _gather_keys_finish (the receive may still be in flight).
+        K-hat (fp16 for the CUDA engine) and V (bf16) travel together as 16-bit words."""
         import torch
+        self._kv_types = (khat_local.dtype, v_local.dtype)
+        if khat_local.dtype != v_local.dtype and khat_local.element_size() == v_local.element_size() == 2:
+            khat_local, v_local = khat_local.view(torch.int16), v_local.view(torch.int16)
         kv = torch.stack([khat_local, v_local], 1)                      # [n, 2, Hkv, D]
         send = [kv.index_select(0, self._idx(("send", dst), self.send_idx[dst], kv.device))
                 for dst in range(self.world)]
@@ -420,7 +434,11 @@ class ContextParallelAttention:
             rem = cat.index_select(0, self._idx("recv", self.recv_order, kv.device))
         else:
             rem = kv.new_zeros((0,) + tuple(kv.shape[1:]))
-        return rem[:, 0], rem[:, 1]
+        kt, vt = self._kv_types
+        rk, rv = rem[:, 0].contiguous(), rem[:, 1].contiguous()
+        if rk.dtype != kt:
+            rk, rv = rk.view(kt), rv.view(vt)
+        return rk, rv
 
     def _cache_grads(self, dkc, dvc, ncl, like):
         """Gradients of the global cache: this rank's rows scattered, summed over ranks."""
@@ -470,25 +488,27 @@ class ContextParallelAttention:
         return dk, dv
 
     def _local_cache(self, k_cache, v_cache, rk, rv):
+        """Cache rows of the local problem: the global cache rows it needs, then the
+        borrowed rows; keys in the type of this rank's K-hat (the engine's cache type)."""
         import torch
         rows = torch.as_tensor(self.local.cache_rows, dtype=torch.long, device=rk.device)
         if len(self.local.cache_rows):
-            kc, vc = k_cache.index_select(0, rows), v_cache.index_select(0, rows)
+            kc, vc = k_cache.index_select(0, rows).to(rk.dtype), v_cache.index_select(0, rows)
             return torch.cat([kc, rk], 0), torch.cat([vc, rv], 0)
         return rk, rv
 
-    def _held_cache(self, k_cache, v_cache):
+    def _held_cache(self, k_cache, v_cache, key_dtype):
         import torch
         if not len(self.local.cache_rows):
             return None, None
         rows = torch.as_tensor(self.local.cache_rows, dtype=torch.long, device=k_cache.device)
-        return k_cache.index_select(0, rows), v_cache.index_select(0, rows)
+        return k_cache.index_select(0, rows).to(key_dtype), v_cache.index_select(0, rows)
 
     def forward(self, q_local, k_local, v_local, k_cache=None, v_cache=None, q_gain=None, k_gain=None):
         khat = self.plan.k_prologue(k_local, k_gain)
         if self.overlap:
             handle = self._gather_keys_start(khat, v_local)
-            kc_h, vc_h = self._held_cache(k_cache, v_cache)
+            kc_h, vc_h = self._held_cache(k_cache, v_cache, khat.dtype)
             o_h, l_h = self.plan_held.fwd(q_local, k_local, v_local, kc_h, vc_h, q_gain=q_gain, k_gain=k_gain)
             rk, rv = self._gather_keys_finish(handle)
             o_b, l_b = self.plan_borrowed.fwd(q_local, k_local, v_local, rk, rv, q_gain=q_gain, k_gain=k_gain)

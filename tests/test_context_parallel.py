@@ -401,3 +401,44 @@ def test_cuda_split_by_key_location_equals_unsplit(name):
     assert (rem_k - gf[3][ncl:]).abs().max().item() <= 1e-2 and (rem_v - gf[4][ncl:]).abs().max().item() <= 1e-2
     if ncl:
         assert (dkc - gf[3][:ncl]).abs().max().item() <= 1e-2 and (dvc - gf[4][:ncl]).abs().max().item() <= 1e-2
+
+
+def test_exchange_keeps_the_key_and_value_types():
+    """K-hat in fp16 (the CUDA engine's cache-key type) and V in bf16 travel together and
+    come back with their own types and bits (one rank: the exchange is a local copy)."""
+    w = W.WORKLOADS["packed_replica"]
+
+    class Strict:
+        """Stands in for the CUDA plan's type checks (no computation)."""
+        def __init__(self, *a, **k):
+            pass
+
+    att = CP.ContextParallelAttention(None, 0, 1, w.hq, w.hkv, w.d, w.videos_array(), w.num_cache_keys,
+                                      w.slices_array(), engine=Strict)
+    n = len(att.local.tokens)
+    g = torch.Generator().manual_seed(3)
+    kh = torch.randn((n, w.hkv, w.d), generator=g).to(torch.float16)
+    v = torch.randn((n, w.hkv, w.d), generator=g).to(torch.bfloat16)
+    rk, rv = att._gather_keys(kh, v)
+    assert rk.dtype == torch.float16 and rv.dtype == torch.bfloat16
+    assert rk.is_contiguous() and rv.is_contiguous()
+    assert rk.shape[0] == len(att.local.remote_rows) == 0
+    # with rows to move: a 2-rank plan's send rows of rank 0, exchanged with itself
+    cp = CP.ContextParallelPlan(2, w.videos_array(), w.num_cache_keys, w.slices_array())
+    att2 = CP.ContextParallelAttention(None, 1, 2, w.hq, w.hkv, w.d, w.videos_array(), w.num_cache_keys,
+                                       w.slices_array(), engine=Strict)
+    att2.world = 1                      # emulate the exchange as a local copy of what rank 0 sends
+    own = att2.local.tokens
+    assert len(cp.send_rows[1][0]) > 0
+    att2.send_idx = [np.searchsorted(own, cp.send_rows[1][0])]
+    att2.recv_counts = [len(cp.send_rows[1][0])]
+    att2.recv_order = np.arange(len(cp.send_rows[1][0]))
+    import dataclasses
+    att2.local = dataclasses.replace(att2.local, remote_rows=np.asarray(cp.send_rows[1][0]))
+    kh2 = torch.randn((len(own), w.hkv, w.d), generator=g).to(torch.float16)
+    v2 = torch.randn((len(own), w.hkv, w.d), generator=g).to(torch.bfloat16)
+    rk2, rv2 = att2._gather_keys(kh2, v2)
+    idx = torch.as_tensor(att2.send_idx[0])
+    assert rk2.dtype == torch.float16 and rv2.dtype == torch.bfloat16
+    assert torch.equal(rk2.view(torch.int16), kh2.index_select(0, idx).view(torch.int16))
+    assert torch.equal(rv2.view(torch.int16), v2.index_select(0, idx).view(torch.int16))
