@@ -313,6 +313,20 @@ def run_ours(a):
     value = flops_step_total * a.steps / (elapsed_ms * 1e-3) / 1e12
     tokens_per_s = w.nq * a.steps / (elapsed_ms * 1e-3)
 
+    # ---- host cost of moving a compiled plan to the next window position (the per-step
+    #      cost of a KV-range stage schedule whose layouts are compiled once and reused)
+    vid0 = np.asarray(w.videos_array(), np.int32).reshape(-1, 5)
+    moves = []
+    for i in range(1, 6):
+        vmov = vid0.copy()
+        vmov[:, 4] += i * int(vid0[0, 1])          # one chunk of frames later per step
+        t_m = time.perf_counter()
+        plan.update_positions(vmov, stream=stream)
+        moves.append(1e3 * (time.perf_counter() - t_m))
+    plan.update_positions(vid0, stream=stream)
+    torch.cuda.synchronize()
+    stage_switch_ms = statistics.median(moves)
+
     # ---- end to end through the public API: pinned host inputs -> device -> fwd -> host
     e2e = None
     if a.e2e_steps > 0:
@@ -458,7 +472,8 @@ def run_ours(a):
                        "d": w.d, "visible_pairs_per_head": pairs,
                        "parallelism": f"head-parallel x{world}" if world > 1 else "1 GPU",
                        "l2": "inputs larger than L2 (Q 1.06 GB, K/V images 0.4 GB, O 1.06 GB)",
-                       "plan_compile_ms": plan_ms, "tokens_per_s": tokens_per_s,
+                       "plan_compile_ms": plan_ms, "plan_move_ms": stage_switch_ms,
+                       "tokens_per_s": tokens_per_s,
                        "pct_peak_sustained": 100 * value / peak_sus / world,
                        "pct_peak_burst": 100 * value / peak_burst / world,
                        "fwd_kernel_tflops": fwd_tflops, "bwd_kernel_tflops": bwd_tflops,
