@@ -27,6 +27,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "kernels.hpp"
 #include "prologue.cuh"
@@ -49,6 +50,8 @@ struct KVArgs {
     int64_t nc, nk, nkt;
     int hkv;
     float eps;
+    int prologue;  // 0: keys given post-prologue (BCA_NO_PROLOGUE)
+    int kc_f16;    // cache keys are fp16 (BCA_CACHE_K_FP16)
     __half *kimg;
     __nv_bfloat16 *vimg;
     // e4m3 images (plans with BCA_FWD_FP8_E4M3)
@@ -72,6 +75,7 @@ struct FwdArgs {
     const uint32_t *masks;
     int64_t nq, nkt;
     int hq, hkv;
+    int prologue;       // 0: queries given post-prologue (BCA_NO_PROLOGUE)
     float eps, qscale;  // qscale = log2(e) / sqrt(D)
     int o_fp32;
     void *o;
@@ -103,12 +107,12 @@ __global__ void __launch_bounds__(128) kv_image_kernel(KVArgs a) {
 
     float x[D];
     if (key < a.nc) {
-        load_row_bf16<D>(a.kc + ((size_t)key * a.hkv + g) * D, x);
+        load_row_16<D>(a.kc + ((size_t)key * a.hkv + g) * D, a.kc_f16 != 0, x);
     } else if (key < a.nk) {
         const int64_t n = key - a.nc;
         load_row_bf16<D>(a.k + ((size_t)n * a.hkv + g) * D, x);
         qk_prologue<D>(x, __ldg(a.pos + n), a.k_gain, a.rope, a.axis_off0, a.axis_off1, a.axis_off2, a.eps,
-                       1.0f);
+                       1.0f, a.prologue != 0);
     } else {
 #pragma unroll
         for (int d = 0; d < D; ++d) x[d] = 0.f;
@@ -200,12 +204,12 @@ __global__ void __launch_bounds__(128) kv_image8_kernel(KVArgs a) {
 
     float x[D];
     if (key < a.nc) {
-        load_row_bf16<D>(a.kc + ((size_t)key * a.hkv + g) * D, x);
+        load_row_16<D>(a.kc + ((size_t)key * a.hkv + g) * D, a.kc_f16 != 0, x);
     } else if (key < a.nk) {
         const int64_t n = key - a.nc;
         load_row_bf16<D>(a.k + ((size_t)n * a.hkv + g) * D, x);
         qk_prologue<D>(x, __ldg(a.pos + n), a.k_gain, a.rope, a.axis_off0, a.axis_off1, a.axis_off2, a.eps,
-                       1.0f);
+                       1.0f, a.prologue != 0);
     } else {
 #pragma unroll
         for (int d = 0; d < D; ++d) x[d] = 0.f;
@@ -316,7 +320,10 @@ __device__ __forceinline__ bool warp_wait_or_abort(uint32_t bar, uint32_t parity
     return __all_sync(0xffffffffu, ok);
 }
 
-template <int D, bool F8>
+// NH: query heads per work item, 2 (their softmax warps 4-7 and 8-11 share each K/V tile)
+// or 1 for an odd group size (warps 8-11 idle).  A compile-time count keeps the MMA
+// issuer's per-tile loop over heads unrolled.
+template <int D, bool F8, int NH>
 __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
     using L = FwdSmem<D, F8>;
     constexpr int DPAD = L::DPAD;
@@ -398,7 +405,7 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0 && n > 0) {
             bool ok = wait_or_abort(bar(L::B_Q_READY + 0), 0, a.status, abort_flag, a.timeout_ns) &&
-                      wait_or_abort(bar(L::B_Q_READY + 1), 0, a.status, abort_flag, a.timeout_ns) &&
+                      (NH < 2 || wait_or_abort(bar(L::B_Q_READY + 1), 0, a.status, abort_flag, a.timeout_ns)) &&
                       wait_or_abort(bar(L::B_KV_FULL + 0), 0, a.status, abort_flag, a.timeout_ns);
             tc_fence_after();
             // Both operands K-major with no swizzle: a core matrix is 8 rows x 16 bytes (8
@@ -430,7 +437,7 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
                 }
             };
             if (ok) {
-                for (int s = 0; s < 2; ++s) {
+                for (int s = 0; s < NH; ++s) {
                     issue_s(s, 0);
                     mma_commit(bar(L::B_S_FULL + s));
                 }
@@ -442,7 +449,7 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
                         ok = wait_or_abort(bar(L::B_KV_FULL + nstage), ((j + 1) / STAGES) & 1, a.status, abort_flag, a.timeout_ns);
                         tc_fence_after();
                     }
-                    for (int s = 0; s < 2 && ok; ++s) {
+                    for (int s = 0; s < NH && ok; ++s) {
                         if (more) {
                             ok = wait_or_abort(bar(L::B_S_FREE + s), j & 1, a.status, abort_flag, a.timeout_ns);
                             if (!ok) break;
@@ -464,7 +471,7 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
             if (!mbar_wait(bar(L::B_MMA_DONE), 0, a.timeout_ns)) record_timeout(a.status, abort_flag);
         }
         __syncwarp();
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && (warp - 4) / 4 < NH) {
         // ------------------------------------------------ softmax / prologue / epilogue
         const int slot = (warp - 4) / 4;
         const int quarter = warp % 4;  // TMEM lane quarter this warp may access
@@ -481,7 +488,7 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
             if (live) {
                 load_row_bf16<D>(a.q + ((size_t)qrow * a.hq + h) * D, x);
                 qk_prologue<D>(x, __ldg(a.pos + qrow), a.q_gain, a.rope, a.axis_off0, a.axis_off1, a.axis_off2,
-                               a.eps, F8 ? 1.0f : a.qscale);
+                               a.eps, F8 ? 1.0f : a.qscale, a.prologue != 0);
             } else {
 #pragma unroll
                 for (int d = 0; d < D; ++d) x[d] = 0.f;
@@ -527,9 +534,14 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
                 for (int c = 0; c < 128; ++c)
                     if (!((w4[c / 32] >> (c % 32)) & 1u)) s[c] = -INFINITY;
             }
-            float mx = s[0];
+            // row maximum: four independent chains of three-input maxima (not one chain of
+            // 127 dependent ones)
+            float m4[4] = {fmaxf(s[0], s[1]), fmaxf(s[2], s[3]), fmaxf(s[4], s[5]), fmaxf(s[6], s[7])};
 #pragma unroll
-            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+            for (int c = 8; c < 128; c += 8)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) m4[u] = max3f(m4[u], s[c + 2 * u], s[c + 2 * u + 1]);
+            float mx = max3f(m4[0], m4[1], fmaxf(m4[2], m4[3]));
             if constexpr (F8) mx *= a.qscale;  // S in log2 units (the scale is positive)
             float alpha = 1.f;
             bool rescale = false;
@@ -540,10 +552,26 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
             }
             const float msub = (m_ref == -INFINITY) ? 0.f : m_ref;
             float sum = 0.f;
+            if constexpr (F8) {
 #pragma unroll
-            for (int c = 0; c < 128; ++c) {
-                s[c] = F8 ? ex2(fmaf(s[c], a.qscale, -msub)) : ex2(s[c] - msub);
-                sum += s[c];
+                for (int c = 0; c < 128; ++c) {
+                    s[c] = ex2(fmaf(s[c], a.qscale, -msub));
+                    sum += s[c];
+                }
+            } else {
+                // P = 2^(S - m) in pairs: the subtraction and the row sum (two partial sums)
+                // as paired fp32 instructions
+                float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                const float2 neg = make_float2(-msub, -msub);
+#pragma unroll
+                for (int c = 0; c < 128; c += 2) {
+                    const float2 x = __fadd2_rn(make_float2(s[c], s[c + 1]), neg);
+                    const float2 p = make_float2(ex2(x.x), ex2(x.y));
+                    s[c] = p.x;
+                    s[c + 1] = p.y;
+                    acc[(c >> 1) & 1] = __fadd2_rn(acc[(c >> 1) & 1], p);
+                }
+                sum = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
             }
             l = l * alpha + sum;
 
@@ -666,6 +694,8 @@ int launch_fwd_d(Plan &P, const FwdIO &io, cudaStream_t stream) {
     ka.nkt = P.nkt;
     ka.hkv = P.hkv;
     ka.eps = P.eps;
+    ka.prologue = (P.flags & BCA_NO_PROLOGUE) ? 0 : 1;
+    ka.kc_f16 = (P.flags & BCA_CACHE_K_FP16) ? 1 : 0;
     ka.kimg = kimg;
     ka.vimg = vimg;
     ka.kimg8 = ws8;
@@ -704,6 +734,7 @@ int launch_fwd_d(Plan &P, const FwdIO &io, cudaStream_t stream) {
     fa.nkt = P.nkt;
     fa.hq = P.hq;
     fa.hkv = P.hkv;
+    fa.prologue = (P.flags & BCA_NO_PROLOGUE) ? 0 : 1;
     fa.eps = P.eps;
     fa.qscale = 1.4426950408889634f / sqrtf((float)D);
     fa.o_fp32 = (P.flags & BCA_O_FP32) ? 1 : 0;
@@ -714,8 +745,12 @@ int launch_fwd_d(Plan &P, const FwdIO &io, cudaStream_t stream) {
     fa.skip_loads = (P.flags & BCA_TEST_FORCE_TIMEOUT) ? 1 : 0;
     {
         ProfScope ps(P, BCA_KERNEL_FWD, stream);
-        if (f8) fwd_kernel<D, true><<<(unsigned)P.items.size(), 384, FwdSmem<D, true>::BYTES, stream>>>(fa);
-        else fwd_kernel<D, false><<<(unsigned)P.items.size(), 384, FwdSmem<D, false>::BYTES, stream>>>(fa);
+        const unsigned grid = (unsigned)P.items.size();
+        const bool two = P.heads_per_item == 2;
+        if (f8 && two) fwd_kernel<D, true, 2><<<grid, 384, FwdSmem<D, true>::BYTES, stream>>>(fa);
+        else if (f8) fwd_kernel<D, true, 1><<<grid, 384, FwdSmem<D, true>::BYTES, stream>>>(fa);
+        else if (two) fwd_kernel<D, false, 2><<<grid, 384, FwdSmem<D, false>::BYTES, stream>>>(fa);
+        else fwd_kernel<D, false, 1><<<grid, 384, FwdSmem<D, false>::BYTES, stream>>>(fa);
     }
     if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
     return BCA_OK;
@@ -739,21 +774,20 @@ int prepare_fwd(const Plan &P) {
     auto set = [](const void *f, int bytes) {
         return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
     };
-    bool ok = true;
     const bool f8 = (P.flags & BCA_FWD_FP8_E4M3) != 0;
+    const bool two = P.heads_per_item == 2;
+    auto pick = [&](auto d_c) -> bool {
+        constexpr int D = decltype(d_c)::value;
+        if (f8 && two) return set((const void *)fwd_kernel<D, true, 2>, FwdSmem<D, true>::BYTES);
+        if (f8) return set((const void *)fwd_kernel<D, true, 1>, FwdSmem<D, true>::BYTES);
+        if (two) return set((const void *)fwd_kernel<D, false, 2>, FwdSmem<D, false>::BYTES);
+        return set((const void *)fwd_kernel<D, false, 1>, FwdSmem<D, false>::BYTES);
+    };
+    bool ok = true;
     switch (P.d) {
-        case 24:
-            ok = f8 ? set((const void *)fwd_kernel<24, true>, FwdSmem<24, true>::BYTES)
-                    : set((const void *)fwd_kernel<24, false>, FwdSmem<24, false>::BYTES);
-            break;
-        case 32:
-            ok = f8 ? set((const void *)fwd_kernel<32, true>, FwdSmem<32, true>::BYTES)
-                    : set((const void *)fwd_kernel<32, false>, FwdSmem<32, false>::BYTES);
-            break;
-        case 48:
-            ok = f8 ? set((const void *)fwd_kernel<48, true>, FwdSmem<48, true>::BYTES)
-                    : set((const void *)fwd_kernel<48, false>, FwdSmem<48, false>::BYTES);
-            break;
+        case 24: ok = pick(std::integral_constant<int, 24>{}); break;
+        case 32: ok = pick(std::integral_constant<int, 32>{}); break;
+        case 48: ok = pick(std::integral_constant<int, 48>{}); break;
         default: return BCA_ERR_UNSUPPORTED;
     }
     return ok ? BCA_OK : BCA_ERR_CUDA;
