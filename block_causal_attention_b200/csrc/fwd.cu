@@ -534,14 +534,9 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
                 for (int c = 0; c < 128; ++c)
                     if (!((w4[c / 32] >> (c % 32)) & 1u)) s[c] = -INFINITY;
             }
-            // row maximum: four independent chains of three-input maxima (not one chain of
-            // 127 dependent ones)
-            float m4[4] = {fmaxf(s[0], s[1]), fmaxf(s[2], s[3]), fmaxf(s[4], s[5]), fmaxf(s[6], s[7])};
+            float mx = s[0];
 #pragma unroll
-            for (int c = 8; c < 128; c += 8)
-#pragma unroll
-                for (int u = 0; u < 4; ++u) m4[u] = max3f(m4[u], s[c + 2 * u], s[c + 2 * u + 1]);
-            float mx = max3f(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
             if constexpr (F8) mx *= a.qscale;  // S in log2 units (the scale is positive)
             float alpha = 1.f;
             bool rescale = false;
@@ -552,26 +547,10 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
             }
             const float msub = (m_ref == -INFINITY) ? 0.f : m_ref;
             float sum = 0.f;
-            if constexpr (F8) {
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    s[c] = ex2(fmaf(s[c], a.qscale, -msub));
-                    sum += s[c];
-                }
-            } else {
-                // P = 2^(S - m) in pairs: the subtraction and the row sum (two partial sums)
-                // as paired fp32 instructions
-                float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-                const float2 neg = make_float2(-msub, -msub);
-#pragma unroll
-                for (int c = 0; c < 128; c += 2) {
-                    const float2 x = __fadd2_rn(make_float2(s[c], s[c + 1]), neg);
-                    const float2 p = make_float2(ex2(x.x), ex2(x.y));
-                    s[c] = p.x;
-                    s[c + 1] = p.y;
-                    acc[(c >> 1) & 1] = __fadd2_rn(acc[(c >> 1) & 1], p);
-                }
-                sum = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
+            for (int c = 0; c < 128; ++c) {
+                s[c] = F8 ? ex2(fmaf(s[c], a.qscale, -msub)) : ex2(s[c] - msub);
+                sum += s[c];
             }
             l = l * alpha + sum;
 
