@@ -842,6 +842,7 @@ struct DqPassArgs {
     float *dqacc;
     int *status;
     uint64_t timeout_ns;
+    int skip_loads;  // failure-detection test: issue no loads, so every wait runs out
 };
 
 template <int D>
@@ -909,7 +910,7 @@ __global__ void __launch_bounds__(384, 1) bwd_dq_pass_kernel(DqPassArgs a) {
     };
 
     if (warp == 0) {
-        if (lane == 0 && n > 0) {
+        if (lane == 0 && n > 0 && !a.skip_loads) {
             const size_t qtile = ((size_t)h * a.nqt + qt) * (128 * DPAD);
             mbar_arrive_expect_tx(bar(L::B_QD), 2 * L::TILE);
             bulk_g2s(sbase + L::OFF_Q, a.qimg16 + qtile, L::TILE, bar(L::B_QD));
@@ -1317,6 +1318,7 @@ int launch_bwd_d(Plan &P, const BwdIO &io, cudaStream_t stream) {
         qa.dqacc = dqacc;
         qa.status = P.d_status;
         qa.timeout_ns = ba.timeout_ns;
+        qa.skip_loads = ba.skip_loads;
         ProfScope ps(P, BCA_KERNEL_BWD_DQ_PASS, stream);
         bwd_dq_pass_kernel<D><<<(unsigned)(P.items.size() * P.heads_per_item), 384, DqSmem<D>::BYTES, stream>>>(qa);
         if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;

@@ -375,6 +375,11 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
     tc_fence_after();
     const uint32_t tbase = *tmem_ptr;
 
+    // Registers: 384 threads x 168 at launch.  The producer / MMA warpgroup (warps 0-3) needs
+    // few and gives them up (96), the softmax warpgroups take 184 (128 x 96 + 256 x 184 =
+    // 59,392 <= 64,512), which removes most of their spills.  Each warpgroup executes its
+    // instruction together (warps 0-3 here, the softmax warpgroup at the top of its branch).
+    if (warp < 4) regs_dec<96>();
     if (warp == 0) {
         // ------------------------------------------------ producer: K/V tiles
         if (lane == 0 && n > 0 && !a.skip_loads) {
@@ -472,6 +477,7 @@ __global__ void __launch_bounds__(384, 1) fwd_kernel(FwdArgs a) {
         }
         __syncwarp();
     } else if (warp >= 4 && (warp - 4) / 4 < NH) {
+        regs_inc<184>();
         // ------------------------------------------------ softmax / prologue / epilogue
         const int slot = (warp - 4) / 4;
         const int quarter = warp % 4;  // TMEM lane quarter this warp may access

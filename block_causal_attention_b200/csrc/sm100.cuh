@@ -273,6 +273,18 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&a)[N], uint32_t (&b
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// ---------------------------------------------------------------- registers
+
+// Per-warpgroup register budget (setmaxnreg): executed by all four warps of a warpgroup.
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- math
 
 __device__ __forceinline__ float ex2(float x) {

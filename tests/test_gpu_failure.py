@@ -56,3 +56,19 @@ def test_forced_timeout_in_the_backward_is_reported_and_context_stays_usable():
                                              w.slices_array(), w.hq, w.hkv)
     for a, b in ((dq, rq), (dk, rk), (dv, rv)):
         assert np.abs(a.double().cpu().numpy() - b).max() < 1e-2
+
+
+def test_forced_timeout_in_the_deterministic_dq_pass_is_reported():
+    """The deterministic dQ pass waits with the same bounded waits (loads withheld too)."""
+    w = W.WORKLOADS["tiny"]
+    x = W.make_inputs(w, "cuda", with_grad=True)
+    good = _plan(w)
+    o, lse = good.fwd(x["q"], x["k"], x["v"])
+    bad = _plan(w, test_force_timeout=True, dq_deterministic=True)
+    bad.bwd(x["q"], x["k"], x["v"], None, None, o, lse, x["do"])
+    torch.cuda.synchronize()
+    assert bad.status() == _abi.BCA_ERR_DEVICE_TIMEOUT
+    assert bad.status() == _abi.BCA_OK
+    good.bwd(x["q"], x["k"], x["v"], None, None, o, lse, x["do"])
+    torch.cuda.synchronize()
+    assert good.status() == _abi.BCA_OK

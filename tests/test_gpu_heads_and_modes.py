@@ -157,3 +157,40 @@ def test_fp16_cache_keys_equal_bf16_cache_keys_when_exact():
     pos = oracle.positions(vids)
     ref = oracle.prologue(x["k"].cpu(), pos, (1e4, 1e4, 1e4), 1e-6)
     assert np.abs(kh.double().cpu().numpy() - ref).max() <= 2 ** -11 * np.abs(ref).max()
+
+
+def test_degenerate_problems():
+    """No new tokens (a cache only), rows that see no key at all, and a single token."""
+    f32 = torch.float32
+    # (1) no new token: the forward launches nothing, the backward zeroes the cache gradients
+    hq, hkv, d, nc = 4, 2, 32, 64
+    p = Plan(hq, hkv, d, np.zeros((0, 5), np.int32), nc, np.zeros((0, 5), np.int64))
+    e = lambda *s: torch.empty(s, dtype=torch.bfloat16, device="cuda")
+    kc, vc = W.seeded_normal_bf16(7701, (nc, hkv, d), "cuda"), W.seeded_normal_bf16(7702, (nc, hkv, d), "cuda")
+    o, lse = p.fwd(e(0, hq, d), e(0, hkv, d), e(0, hkv, d), kc, vc)
+    dkc = torch.full((nc, hkv, d), 7.0, dtype=f32, device="cuda")
+    dvc = torch.full((nc, hkv, d), 7.0, dtype=f32, device="cuda")
+    p.bwd(e(0, hq, d), e(0, hkv, d), e(0, hkv, d), kc, vc, o, lse, e(0, hq, d), dk_cache=dkc, dv_cache=dvc)
+    torch.cuda.synchronize()
+    assert p.status() == _abi.BCA_OK and o.numel() == 0
+    assert (dkc == 0).all() and (dvc == 0).all()
+    # (2) an explicit empty slice list: no row sees a key -> O = 0, LSE = -inf, gradients 0
+    vids, _, nc2, x = _problem(7710, 4, 2, 48, C=80)
+    p2 = Plan(4, 2, 48, vids, nc2, np.zeros((0, 5), np.int64))
+    o2, l2 = p2.fwd(x["q"], x["k"], x["v"], x["kc"], x["vc"])
+    g2 = p2.bwd(x["q"], x["k"], x["v"], x["kc"], x["vc"], o2, l2, x["do"])
+    torch.cuda.synchronize()
+    assert p2.status() == _abi.BCA_OK
+    assert (o2 == 0).all() and torch.isneginf(l2).all()
+    for t in g2:
+        assert (t == 0).all()
+    # (3) one token, one key: P = 1 exactly, so O is the token's V row
+    p3 = Plan(4, 2, 48, np.asarray([[1, 1, 1, 1, 0]], np.int32), 0, None)
+    q3, k3, v3 = (W.seeded_normal_bf16(7720 + i, (1, h, 48), "cuda") for i, h in enumerate((4, 2, 2)))
+    o3, l3 = p3.fwd(q3, k3, v3)
+    torch.cuda.synchronize()
+    assert p3.status() == _abi.BCA_OK
+    assert torch.equal(o3, v3.repeat_interleave(2, dim=1))
+    ro, rl = oracle.forward(q3.cpu(), k3.cpu(), v3.cpu(), None, None, np.asarray([[1, 1, 1, 1, 0]], np.int32),
+                            np.asarray([[0, 1, 0, 1, 0]], np.int64), 4, 2)
+    assert np.abs(l3.double().cpu().numpy().T - rl).max() <= 1e-3
