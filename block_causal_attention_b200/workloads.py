@@ -202,10 +202,6 @@ WORKLOADS = {
                        description="4 chunks x 192 (2x8x12), D=24"),
 }
 
-# BASELINE order: config index -> workload name
-CONFIG_ORDER = ["tiny", "b45_infer", "p720_pipelined", "packed_varlen", "long_kvrange"]
-
-
 # ---------------------------------------------------------------------------
 # counter-based N(0,1)->bf16 generator
 # ---------------------------------------------------------------------------
