@@ -299,18 +299,17 @@ def _default_engine(hq, hkv, d, videos, num_cache_keys, slices, rope_base, eps, 
 
 
 def _host_staged(group, t) -> bool:
-    """True when the collectives of `group` cannot take `t` as it is: device tensors on a
-    gloo group (gloo moves host memory) go through host copies, and 16-bit words (which
-    gloo has no type for) travel in pairs as 32-bit words."""
-    import torch
+    """True when the collectives of `group` cannot take `t` where it lives: device tensors
+    on a gloo group (gloo moves host memory) go through host copies."""
     import torch.distributed as dist
-    return dist.get_backend(group) == "gloo" and (t.is_cuda or t.dtype == torch.int16)
+    return t.is_cuda and dist.get_backend(group) == "gloo"
 
 
 def _all_to_all_rows(group, send: List, recv_counts: List[int], row_shape, like, async_op: bool = False):
     """Rows of `send[dst]` go to rank dst; returns the received rows per source rank (and,
     with async_op, the pending work to wait on before reading them).  Rows are moved
-    bit-exactly (as 16-bit integers for 16-bit types)."""
+    bit-exactly: 16-bit rows (an even count of elements per row) travel as 32-bit words,
+    a type every backend has (gloo and NCCL have no 16-bit integer type)."""
     import torch
     import torch.distributed as dist
     world = len(send)
@@ -318,22 +317,17 @@ def _all_to_all_rows(group, send: List, recv_counts: List[int], row_shape, like,
     flat = [s.reshape(-1, width) for s in send]
     sbuf = torch.cat(flat, 0) if flat else like.new_zeros((0, width))
     rbuf = like.new_empty((sum(recv_counts), width))
-    as_int = sbuf.dtype in (torch.bfloat16, torch.float16)
-    sview = sbuf.view(torch.int16) if as_int else sbuf
-    rview = rbuf.view(torch.int16) if as_int else rbuf
+    pack = sbuf.element_size() == 2 and width % 2 == 0
+    sview = sbuf.view(torch.int32) if pack else sbuf
+    rview = rbuf.view(torch.int32) if pack else rbuf
     work = None
     if world == 1:
         rview.copy_(sview)
     elif _host_staged(group, sview):
-        # gloo has no 16-bit integer type: 16-bit rows (an even count per row) travel as
-        # pairs packed into 32-bit words, still bit-exact
-        pack = sview.dtype == torch.int16
-        shost = sview.cpu()
-        shost = shost.view(torch.int32) if pack else shost
-        rhost = torch.empty((rview.shape[0], shost.shape[1]), dtype=shost.dtype)
-        dist.all_to_all_single(rhost, shost, output_split_sizes=list(recv_counts),
+        rhost = torch.empty(rview.shape, dtype=rview.dtype)
+        dist.all_to_all_single(rhost, sview.cpu(), output_split_sizes=list(recv_counts),
                                input_split_sizes=[int(f.shape[0]) for f in flat], group=group)
-        rview.copy_(rhost.view(torch.int16) if pack else rhost)
+        rview.copy_(rhost)
     else:
         work = dist.all_to_all_single(rview, sview, output_split_sizes=list(recv_counts),
                                       input_split_sizes=[int(f.shape[0]) for f in flat], group=group,
