@@ -480,3 +480,34 @@ def test_golden_key_grads_script_equals_the_dense_backward(name):
             want_v = dvc[j, g] if j < nc else dv[j - nc, g]
             assert np.abs(k_dk[a] - want_k).max() <= 1e-12, (g, j)
             assert np.abs(k_dv[a] - want_v).max() <= 1e-12, (g, j)
+
+
+@pytest.mark.parametrize("D", [32, 48])
+def test_row_backward_equals_the_dense_backward(D):
+    """backward_rows (the per-row C backward behind the full-size dQ row samples, through
+    the prologue) gives the dense backward's dq, and attn_bwd_rows its O and LSE, on rows
+    in any order: GQA with a KV cache, a FULL and a CAUSAL slice that overlap, and a row
+    that sees no key (dq = 0).  The dense backward is pinned by central differences."""
+    Hq, Hkv = 4, 2
+    videos = np.asarray([[2, 1, 2, 3, 4]], np.int32)      # 2 chunks of 6 tokens, t0 = 4
+    nq, nc = 12, 6
+    sl = np.asarray([(0, 5, 0, 12, 0), (6, 12, 6, 18, 1), (8, 12, 0, 9, 0)], np.int64)  # row 5 sees nothing
+    q, k, v = _rand((nq, Hq, D)), _rand((nq, Hkv, D)), _rand((nq, Hkv, D))
+    kc, vc, do = _rand((nc, Hkv, D)), _rand((nc, Hkv, D)), _rand((nq, Hq, D))
+    g_q, g_k = RNG.uniform(0.5, 1.5, D), RNG.uniform(0.5, 1.5, D)
+    base = (100.0, 50.0, 20.0)
+    dq, _, _, _, _, O, lse = oracle.backward(q, k, v, kc, vc, do, videos, sl, Hq, Hkv, base=base,
+                                             q_gain=g_q, k_gain=g_k)
+    rows = np.asarray([11, 5, 0, 7, 3, 6], np.int64)
+    dq_r = oracle.backward_rows(q[rows], rows, k, v, kc, vc, do[rows], videos, sl, Hq, Hkv, base=base,
+                                q_gain=g_q, k_gain=g_k)
+    assert np.abs(dq_r - dq[rows]).max() <= 1e-12
+    assert np.all(dq_r[1] == 0.0)
+    pos = oracle.positions(videos)
+    kh = oracle.full_keys(oracle.prologue(k, pos, base, 1e-6, g_k), kc)
+    qh = oracle.prologue(q[rows], pos[rows], base, 1e-6, g_q)
+    _, O_r, lse_r = oracle.attn_bwd_rows(qh, rows, kh, oracle.full_keys(v, vc), do[rows], sl, Hq, Hkv)
+    assert np.abs(O_r - O[rows]).max() <= 1e-12
+    assert np.array_equal(np.isneginf(lse_r), np.isneginf(lse[rows]))
+    fin = np.isfinite(lse_r)
+    assert np.abs(lse_r[fin] - lse[rows][fin]).max() <= 1e-12
